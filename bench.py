@@ -1,0 +1,333 @@
+"""Benchmark of the RotateAttention INT4 forward hot path on B200.
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+the fused prologue (ra_rope_rotate_quant) followed by the INT4 attention
+(ra_attn_int4), on the Wan-14B-480p-like attention shape (B=1, H=40,
+N=32760, D=128, segments 44/42/42, interleaved rotation, 128x64 blocks).
+
+Metric: INT4 attention TOPS = 4 N^2 D H / t, with t the device time of a whole
+step.  Prints one JSON line (rank 0).  See --help for options.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (launched by torch.distributed.run): every rank runs its own
+independent batch (weak scaling, no collective on the data path); the step
+time is the maximum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "INT4 attn TOPS (4N²DH/t) & % INT8 tensor peak at N=32760,H=40,D=128"
+KERNELS_PER_STEP = 5  # rope table, channel reduce, finalize, quantise, attention
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            m = json.load(f)
+        return {"hbm_gbs": float(m["hbm_gbs"]), "bf16_tflops": float(m["bf16_tflops"]),
+                "bf16_tflops_sustained": float(m.get("bf16_tflops_sustained", m["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi during the timed region."""
+
+    def __init__(self, index: int):
+        self.index = index
+        self.samples = []
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+        while not self._stop.is_set():
+            try:
+                out = subprocess.run(["nvidia-smi", "-i", str(self.index), f"--query-gpu={q}",
+                                      "--format=csv,noheader,nounits"], capture_output=True, text=True,
+                                     timeout=5).stdout.strip()
+                if out:
+                    self.samples.append([s.strip() for s in out.split(",")])
+            except Exception:
+                pass
+            self._stop.wait(0.2)
+
+    def __enter__(self):
+        self._t = threading.Thread(target=self._run, daemon=True)
+        self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        self._t.join(timeout=10)
+
+    def summary(self):
+        sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
+        mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in self.samples for i in range(4)
+                          if len(s) > 3 + i and s[3 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+def _workload(name):
+    from synth import inputs as si
+    return si.WORKLOADS[name]
+
+
+def _config(wl, extra=None):
+    rot = {0: "none", 1: "interleaved", 2: "half"}[wl.rot]
+    c = {"workload": f"{wl.name}: B={wl.B} H={wl.H} N={wl.N} (grid {wl.grid[0]}x{wl.grid[1]}x{wl.grid[2]}) "
+                     f"D={wl.D} seg={wl.seg[0]}/{wl.seg[1]}/{wl.seg[2]} rot={rot} blocks {wl.block_q}x{wl.block_k}",
+         "B": wl.B, "H": wl.H, "N": wl.N, "D": wl.D, "seg": list(wl.seg), "rot": rot,
+         "block_q": wl.block_q, "block_k": wl.block_k,
+         "l2": "inputs larger than L2: Q/K/V bf16 = %.2f GB per step" % (3 * wl.B * wl.H * wl.N * wl.D * 2 / 1e9)}
+    if extra:
+        c.update(extra)
+    return c
+
+
+def cpu_baseline(wl, target_s: float = 15.0):
+    """The oracle, as it stands, on a bounded sample of the workload: the
+    prologue of head 0 and the attention of as many 128-row query tiles of head 0
+    as fit in about target_s seconds; value prorated to the metric's unit."""
+    import numpy as np
+    import oracle
+    from synth import inputs as si
+    x = si.make_inputs(wl, heads=(0,))
+    p = oracle.problem(wl)
+    t0 = time.perf_counter()
+    h = oracle.prologue_head(p, x["q"][0, 0], x["k"][0, 0], x["v"][0, 0], x["pos"])
+    t_pro = time.perf_counter() - t0
+    rows = 0
+    t_att = 0.0
+    ntiles = -(-wl.N // 128)
+    tile = 0
+    while t_att < target_s and tile < ntiles:
+        r0 = tile * 128
+        r1 = min(r0 + 128, wl.N)
+        t0 = time.perf_counter()
+        oracle.attention_int4_rows(p, h, r0, r1)
+        t_att += time.perf_counter() - t0
+        rows += r1 - r0
+        tile += max(1, ntiles // 16)
+    t = t_att + t_pro * rows / wl.N
+    ops = 4.0 * rows * wl.N * wl.D
+    return {"value": ops / t / 1e12, "unit": "TOPS", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"head 0 of {wl.name}: prologue of all {wl.N} tokens (prorated to the rows) + "
+                      f"attention of {rows} query rows over all {wl.N} keys; {t:.1f} s of CPU time"}
+
+
+def run_ours(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+
+    import __graft_entry__
+    __graft_entry__.build()
+    import int4_quantized_flashattention_b200 as ra
+    from synth import inputs as si
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = _workload(args.workload)
+    x = si.make_inputs(wl)
+    p = ra.Problem.make(wl.B, wl.H, wl.D, wl.seg, wl.grid, theta=wl.theta, rot=wl.rot,
+                        block_q=wl.block_q, block_k=wl.block_k)
+    host = {n: torch.from_numpy(x[n + "_bits"]).view(torch.bfloat16).pin_memory() for n in ("q", "k", "v")}
+    pos_h = torch.from_numpy(x["pos"]).pin_memory()
+    q, k, v = (host[n].to(dev) for n in ("q", "k", "v"))
+    pos = pos_h.to(dev)
+    ws = torch.empty(ra.workspace_bytes(p), dtype=torch.uint8, device=dev)
+    codes = ra.rope_rotate_quant(p, q, k, v, pos, workspace=ws)
+    out = torch.empty(wl.B, wl.H, wl.N, wl.D, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ra.rope_rotate_quant(p, q, k, v, pos, out=codes, workspace=ws)
+        ra.attn_int4(p, codes, out=out)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if ra.sync_status() != 0:
+        raise RuntimeError("device status not ok after warm-up")
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local_rank) as clk:
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for i in range(args.steps):
+            a, b, c = ev[i]
+            a.record(stream)
+            ra.rope_rotate_quant(p, q, k, v, pos, out=codes, workspace=ws)
+            b.record(stream)
+            ra.attn_int4(p, codes, out=out)
+            c.record(stream)
+        end.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    total_ms = start.elapsed_time(end)
+    pro_ms = [a.elapsed_time(b) for a, b, _ in ev]
+    att_ms = [b.elapsed_time(c) for _, b, c in ev]
+    status = ra.sync_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed region")
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    # end to end through the public API with host buffers: H2D of Q/K/V (pinned),
+    # prologue + attention, D2H of the output, every step
+    out_h = torch.empty(out.shape, dtype=torch.bfloat16).pin_memory()
+    for _ in range(2):
+        for n, t in (("q", q), ("k", k), ("v", v)):
+            t.copy_(host[n], non_blocking=True)
+        step()
+        out_h.copy_(out, non_blocking=True)
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        for n, t in (("q", q), ("k", k), ("v", v)):
+            t.copy_(host[n], non_blocking=True)
+        pos.copy_(pos_h, non_blocking=True)
+        step()
+        out_h.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / args.steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = sum(host[n].numel() * 2 for n in ("q", "k", "v")) + pos_h.numel() * 4
+    d2h = out_h.numel() * 2
+
+    ops = wl.attn_ops()
+    ms_step = total_ms / args.steps
+    value = world * ops / (ms_step * 1e-3) / 1e12
+    pk = _peaks()
+    int8_peak = 2.0 * pk["bf16_tflops"]        # nominal dense int8 / bf16 ratio on B200 = 2
+    att_med = statistics.median(att_ms)
+    pro_med = statistics.median(pro_ms)
+    achieved = ops / (att_med * 1e-3) / 1e12
+    pro_bytes = prologue_bytes(wl)
+    res = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int4", "data": "synthetic (seeded, outlier-structured; no model weights)",
+        "config": _config(wl, {"parallelism": f"independent batch per GPU x{world}"}),
+        "e2e": {"value": round(world * ops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TOPS",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "roofline": {"bound": "tensor", "kernel": "attn_int4_kernel", "achieved": round(achieved, 1),
+                     "peak": round(int8_peak, 1), "unit": "TFLOP/s", "frac": round(achieved / int8_peak, 4),
+                     "peak_source": f"2 x {pk['source']} bf16 burst {pk['bf16_tflops']} TFLOP/s (int8 ops/s)",
+                     "traffic": None},
+        "prologue": {"ms": round(pro_med, 4), "bytes": pro_bytes,
+                     "achieved_gbs": round(pro_bytes / (pro_med * 1e-3) / 1e9, 1),
+                     "peak_gbs": pk["hbm_gbs"], "frac": round(pro_bytes / (pro_med * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
+                     "ratio_to_attention": round(pro_med / att_med, 4)},
+        "attention_ms": round(att_med, 4),
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "clocks": clk.summary(),
+    }
+    return res
+
+
+def prologue_bytes(wl):
+    """Algorithmic bytes of the prologue: Q once, K and V twice (bf16), packed
+    codes, per-token and per-channel scales, K means, V column sums."""
+    B, H, N, D = wl.B, wl.H, wl.N, wl.D
+    el = 2 if wl.dtype == "bf16" else 4
+    reads = (1 + 2 + 2) * B * H * N * D * el
+    nb = -(-N // wl.block_k)
+    writes = 3 * B * H * N * D // 2 + 2 * 4 * B * H * N + 3 * 4 * B * H * D + 4 * B * H * nb * D
+    return reads + writes
+
+
+def run_reference(args):
+    """The oracle as it stands, on the host cores, one bounded sample per step."""
+    wl = _workload(args.workload)
+    import oracle
+    oracle.lib()
+    vals = []
+    base = None
+    for i in range(args.warmup + args.steps):
+        r = cpu_baseline(wl, target_s=args.ref_seconds)
+        if i >= args.warmup:
+            vals.append(r["value"])
+            base = r
+    v = statistics.median(vals)
+    ms = 4.0 * wl.N * wl.N * wl.D * wl.H * wl.B / (v * 1e12) * 1e3
+    return {"metric": METRIC, "value": round(v, 6), "unit": "TOPS", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 1), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int4", "data": "synthetic (seeded, outlier-structured; no model weights)",
+            "config": _config(wl), "impl": "reference",
+            "cpu_baseline": {"value": round(v, 6), "unit": "TOPS", "cores": base["cores"], "kind": "oracle",
+                             "sample": base["sample"]},
+            "e2e": {"value": round(v, 6), "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="wan")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the CPU oracle sample")
+    ap.add_argument("--ref-seconds", type=float, default=10.0, help="CPU seconds per reference sample")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    if world > 1:
+        import datetime
+        import torch
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    try:
+        res = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                res["cpu_baseline"] = cpu_baseline(_workload(args.workload))
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,591 @@
+// INT4 attention forward of RotateAttention on sm_100a (tcgen05 kind::i8).
+//
+// Method (papernotes page, flowchart D-F and key design 2):
+//   S_ij = (S_int_ij * s_k[j]) * (s_q[i] / sqrt(D)),  S_int = sum_d q4 k4 (exact)
+//   online softmax over key blocks of block_k keys with the running row max m
+//   P codes c_ij = clamp(rint(15 exp(S_ij - m)), 0, 15) - 8
+//   acc_t = sum_j (c_ij + 8) v4_jd  (= sum_j c_ij v4_jd + 8 colsum_t: the
+//           zero-point correction folded into the integer accumulator)
+//   O = sum_t alpha-chain (s_v/15) acc_t / sum_t alpha-chain sum_j (c_ij+8)/15
+//
+// B200 design:
+//   * No 4-bit integer MMA exists on sm_100a; packed nibbles are widened to s8
+//     in shared memory (as 16 x code: the high nibble in place, the low nibble
+//     shifted up), which scales S_int by 256 and acc by 16, both exact powers
+//     of two folded into the fp32 scales.  The widened K dimension of Q and K
+//     follows the same channel permutation, which leaves S_int unchanged.
+//   * QK^T: tcgen05.mma kind::i8, A = Q (smem), B = K (smem), D = S (s32, TMEM).
+//   * P codes are produced as unsigned bytes c + 8 in [0, 15] and stored into
+//     TMEM over the S columns they came from; P.V is a TMEM-A kind::i8 MMA
+//     (A u8, B s8, V MN-major), so the accumulator is sum_j (c_ij + 8) v_jd.
+//   * The s32 P.V accumulator stays in TMEM across key blocks and is folded
+//     into the fp32 output (registers) only when the running maximum of a row
+//     of the warp grows, or when its magnitude bound requires it.  The
+//     accumulator is pre-loaded with the bits of 1.5 * 2^23 so that it reads
+//     back as a float with one subtraction.
+//   * Two 128-row query tiles per CTA share every K/V tile; warp roles:
+//     TMA producer, MMA issuer, two widening warps, two softmax warpgroups
+//     (one thread per query row).  Persistent CTAs, one per SM.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "ra_common.cuh"
+#include "ra_internal.h"
+
+namespace ra {
+namespace {
+
+__device__ uint32_t g_attn_status = 0;
+
+constexpr int kThreads = 384;
+constexpr int kRows = 128;          // query rows per tile = MMA M
+constexpr int kTiles = 2;           // query tiles per CTA
+constexpr uint32_t kMagic = 0x4B400000u;  // bits of 1.5 * 2^23
+constexpr float kMagicF = 12582912.0f;
+
+template <int D, int BN>
+struct Cfg {
+  static constexpr int kPackRow = D / 2;                // packed bytes per row
+  static constexpr int kKeysPV = BN < 32 ? 32 : BN;     // P.V MMA K extent
+  static constexpr int kPS = 4, kKS = 4, kVS = 4;       // pipeline stages
+  static constexpr int kQBytes = kRows * D;             // one widened Q tile
+  static constexpr int kQPkBytes = kRows * kPackRow;
+  static constexpr int kKwBytes = BN * D;
+  static constexpr int kVwBytes = kKeysPV * D;
+  static constexpr int kPkHalf = BN * kPackRow;         // packed K (or V) of one block
+  // shared-memory map (bytes from a 1024-aligned base)
+  static constexpr int oQ = 0;
+  static constexpr int oQPk = oQ + kTiles * kQBytes;
+  static constexpr int oKw = oQPk + kTiles * kQPkBytes;
+  static constexpr int oVw = oKw + kKS * ((kKwBytes + 1023) / 1024) * 1024;
+  static constexpr int oPk = oVw + kVS * ((kVwBytes + 1023) / 1024) * 1024;
+  static constexpr int oKsc = oPk + kPS * 2 * kPkHalf;
+  static constexpr int oBar = oKsc + kKS * BN * 4;
+  static constexpr int kNumBars = 4 + 2 * kPS + 2 * kKS + 2 * kVS + 4 + 4 + 2 + 1;
+  static constexpr int oMisc = oBar + kNumBars * 8;
+  static constexpr int kSmem = oMisc + 16 + 1024;       // + alignment slack
+  static constexpr int kKwStride = ((kKwBytes + 1023) / 1024) * 1024;
+  static constexpr int kVwStride = ((kVwBytes + 1023) / 1024) * 1024;
+  static constexpr uint32_t kSwz = D == 128 ? kSwizzle128B : kSwizzle64B;
+  static constexpr uint32_t kIdescQK = instr_desc(kCfmtS32, 1, 1, 0, 0, kRows, BN);
+  static constexpr uint32_t kIdescPV = instr_desc(kCfmtS32, 0, 1, 0, 1, kRows, D);
+  static_assert(D == 64 || D == 128, "head dim");
+  static_assert(BN == 16 || BN == 32 || BN == 64, "block_k");
+};
+
+struct Bars {
+  uint64_t* qpk_full; uint64_t* qpk_empty; uint64_t* q_full; uint64_t* q_free;
+  uint64_t* pk_full; uint64_t* pk_empty;
+  uint64_t* kw_full; uint64_t* kw_empty;
+  uint64_t* vw_full; uint64_t* vw_empty;
+  uint64_t* s_full;   // [tile][buf]
+  uint64_t* p_full;   // [tile][buf]
+  uint64_t* pv_done;  // [tile]
+  uint64_t* drain;
+};
+
+struct AttnParams {
+  int N, BH, nblocks, npairs, nitems;
+  float inv_sqrt_d;
+  const float* sq;
+  const float* sk;
+  const float* sv;
+  __nv_bfloat16* out;
+  float* lse;
+  // dump variant
+  int dump_bh, dump_tile;
+  int32_t* dump_s;
+  int8_t* dump_p;
+  int32_t* dump_acc;
+};
+
+// Widens one 16-byte chunk of packed codes (32 channels) into two 16-byte
+// chunks of s8 holding 16 x code: low nibbles first, then high nibbles.
+__device__ __forceinline__ void widen_chunk(const uint8_t* src, uint8_t* dst_lo, uint8_t* dst_hi) {
+  const uint4 w = *reinterpret_cast<const uint4*>(src);
+  uint4 lo, hi;
+  lo.x = (w.x << 4) & 0xF0F0F0F0u; hi.x = w.x & 0xF0F0F0F0u;
+  lo.y = (w.y << 4) & 0xF0F0F0F0u; hi.y = w.y & 0xF0F0F0F0u;
+  lo.z = (w.z << 4) & 0xF0F0F0F0u; hi.z = w.z & 0xF0F0F0F0u;
+  lo.w = (w.w << 4) & 0xF0F0F0F0u; hi.w = w.w & 0xF0F0F0F0u;
+  *reinterpret_cast<uint4*>(dst_lo) = lo;
+  *reinterpret_cast<uint4*>(dst_hi) = hi;
+}
+
+// Widens `rows` packed rows (D/2 bytes each, linear) into a swizzled tile of
+// D-byte rows; threads [tid0, tid0 + nthr) share the work.
+template <int D>
+__device__ __forceinline__ void widen_tile(const uint8_t* pk, uint8_t* wide, int rows, int tid, int nthr) {
+  constexpr int kPc = D / 32;  // packed 16-byte chunks per row
+  for (int idx = tid; idx < rows * kPc; idx += nthr) {
+    const int r = idx / kPc, pc = idx % kPc;
+    widen_chunk(pk + r * (D / 2) + pc * 16, wide + swz_offset(r, 2 * pc, D), wide + swz_offset(r, 2 * pc + 1, D));
+  }
+}
+
+// Widened position n (0..D-1) of a row -> channel.
+__host__ __device__ constexpr int wide_to_dim(int n) {
+  return (n & ~31) + 8 * ((n & 15) >> 2) + 2 * (n & 3) + ((n >> 4) & 1);
+}
+
+__device__ __forceinline__ float max3(float a, float b, float c) { return fmaxf(a, fmaxf(b, c)); }
+
+__device__ __forceinline__ void set_status(uint32_t bits) { atomicOr(&g_attn_status, bits); }
+
+template <int D, int BN, bool DUMP>
+__global__ void __launch_bounds__(kThreads, 1)
+attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_v, const AttnParams prm) {
+  using C = Cfg<D, BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::oBar);
+  Bars B;
+  {
+    uint64_t* b = bar;
+    B.qpk_full = b++; B.qpk_empty = b++; B.q_full = b++; B.q_free = b++;
+    B.pk_full = b; b += C::kPS; B.pk_empty = b; b += C::kPS;
+    B.kw_full = b; b += C::kKS; B.kw_empty = b; b += C::kKS;
+    B.vw_full = b; b += C::kVS; B.vw_empty = b; b += C::kVS;
+    B.s_full = b; b += 4; B.p_full = b; b += 4; B.pv_done = b; b += 2; B.drain = b; b += 1;
+  }
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::oMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::oMisc + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(B.qpk_full, 1); mbar_init(B.qpk_empty, 2); mbar_init(B.q_full, 2); mbar_init(B.q_free, 1);
+    for (int s = 0; s < C::kPS; ++s) { mbar_init(B.pk_full + s, 1); mbar_init(B.pk_empty + s, 2); }
+    for (int s = 0; s < C::kKS; ++s) { mbar_init(B.kw_full + s, 2); mbar_init(B.kw_empty + s, 1 + 8); }
+    for (int s = 0; s < C::kVS; ++s) { mbar_init(B.vw_full + s, 2); mbar_init(B.vw_empty + s, 1); }
+    for (int s = 0; s < 4; ++s) { mbar_init(B.s_full + s, 1); mbar_init(B.p_full + s, 4); }
+    mbar_init(B.pv_done + 0, 1); mbar_init(B.pv_done + 1, 1); mbar_init(B.drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_holder;
+
+  const int nb = prm.nblocks;
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
+    if (warp == 0) {
+      // ------------------------------------------------------------ TMA producer
+      if (lane == 0) {
+        uint32_t g = 0, li = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; item < prm.nitems && ok; item += gridDim.x, ++li) {
+          const int bh = item / prm.npairs, pair = item % prm.npairs;
+          ok = mbar_wait(B.qpk_empty, (li & 1) ^ 1, abort_flag);
+          if (!ok) break;
+          mbar_arrive_expect_tx(B.qpk_full, kTiles * C::kQPkBytes);
+          for (int tt = 0; tt < kTiles; ++tt)
+            tma_load_3d(smem + C::oQPk + tt * C::kQPkBytes, &tm_q, B.qpk_full, 0, pair * 2 * kRows + tt * kRows, bh);
+          for (int t = 0; t < nb; ++t, ++g) {
+            const int s = g % C::kPS;
+            ok = mbar_wait(B.pk_empty + s, ((g / C::kPS) & 1) ^ 1, abort_flag);
+            if (!ok) break;
+            mbar_arrive_expect_tx(B.pk_full + s, 2 * C::kPkHalf);
+            uint8_t* dst = smem + C::oPk + s * 2 * C::kPkHalf;
+            tma_load_3d(dst, &tm_k, B.pk_full + s, 0, t * BN, bh);
+            tma_load_3d(dst + C::kPkHalf, &tm_v, B.pk_full + s, 0, t * BN, bh);
+          }
+        }
+        // Wait (bounded) for the copies of the last stages to land.
+        for (uint32_t k = (g > (uint32_t)C::kPS ? g - C::kPS : 0); k < g; ++k) {
+          uint64_t* fb = B.pk_full + (k % C::kPS);
+          uint32_t it = 0;
+          while (!mbar_try_wait(fb, (k / C::kPS) & 1) && ++it < kSpinLimit) {}
+        }
+        if (!ok) set_status(kStatusTimeout);
+      }
+    } else if (warp == 1) {
+      // ------------------------------------------------------------ MMA issuer
+      if (lane == 0) {
+        const uint32_t sQ = smem_u32(smem + C::oQ);
+        const uint32_t sKw = smem_u32(smem + C::oKw);
+        const uint32_t sVw = smem_u32(smem + C::oVw);
+        uint32_t g = 0, li = 0;
+        bool ok = true;
+        auto issue_pv = [&](uint32_t gg) -> bool {
+          const int vs = gg % C::kVS;
+          if (!mbar_wait(B.vw_full + vs, (gg / C::kVS) & 1, abort_flag)) return false;
+          const uint32_t buf = gg & 1;
+          for (int tt = 0; tt < kTiles; ++tt) {
+            if (!mbar_wait(B.p_full + tt * 2 + buf, (gg >> 1) & 1, abort_flag)) return false;
+            tc_fence_after();
+            const uint32_t tP = tbase + tt * 256 + buf * 64;
+            const uint32_t tA = tbase + tt * 256 + 128;
+#pragma unroll
+            for (int kk = 0; kk < C::kKeysPV / 32; ++kk) {
+              const uint64_t bdesc = smem_desc(sVw + vs * C::kVwStride + kk * 32 * D, 8 * D * (C::kKeysPV / 8),
+                                               8 * D, C::kSwz);
+              mma_i8_ts(tA, tP + kk * 8, bdesc, C::kIdescPV, 1);
+            }
+            mma_commit(B.pv_done + tt);
+          }
+          mma_commit(B.vw_empty + vs);
+          return true;
+        };
+        for (int item = blockIdx.x; item < prm.nitems && ok; item += gridDim.x, ++li) {
+          ok = mbar_wait(B.q_full, li & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          for (int t = 0; t < nb && ok; ++t, ++g) {
+            const int ks = g % C::kKS;
+            ok = mbar_wait(B.kw_full + ks, (g / C::kKS) & 1, abort_flag);
+            if (!ok) break;
+            tc_fence_after();
+            const uint32_t buf = g & 1;
+            for (int tt = 0; tt < kTiles; ++tt) {
+              const uint32_t tS = tbase + tt * 256 + buf * 64;
+#pragma unroll
+              for (int kk = 0; kk < D / 32; ++kk) {
+                const uint64_t adesc = smem_desc(sQ + tt * C::kQBytes + kk * 32, 16, 8 * D, C::kSwz);
+                const uint64_t bdesc = smem_desc(sKw + ks * C::kKwStride + kk * 32, 16, 8 * D, C::kSwz);
+                mma_i8_ss(tS, adesc, bdesc, C::kIdescQK, kk > 0 ? 1u : 0u);
+              }
+              mma_commit(B.s_full + tt * 2 + buf);
+            }
+            mma_commit(B.kw_empty + ks);
+            if (t == nb - 1) mma_commit(B.q_free);
+            if (t > 0) ok = issue_pv(g - 1);
+          }
+          if (ok) ok = issue_pv(g - 1);
+        }
+        // Drain: every MMA issued so far has completed before TMEM is released.
+        mma_commit(B.drain);
+        uint32_t it = 0;
+        while (!mbar_try_wait(B.drain, 0) && ++it < kSpinLimit) {}
+        if (!ok) set_status(kStatusTimeout);
+      }
+    } else {
+      // ------------------------------------------------------------ widening warps
+      const int wt = threadIdx.x - 64;  // 0..63
+      uint32_t g = 0, li = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < prm.nitems && ok; item += gridDim.x, ++li) {
+        const int bh = item / prm.npairs;
+        if (!(ok = mbar_wait(B.qpk_full, li & 1, abort_flag))) break;
+        if (!(ok = mbar_wait(B.q_free, (li & 1) ^ 1, abort_flag))) break;
+        for (int tt = 0; tt < kTiles; ++tt)
+          widen_tile<D>(smem + C::oQPk + tt * C::kQPkBytes, smem + C::oQ + tt * C::kQBytes, kRows, wt, 64);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) { mbar_arrive(B.qpk_empty); mbar_arrive(B.q_full); }
+        for (int t = 0; t < nb; ++t, ++g) {
+          const int s = g % C::kPS, ks = g % C::kKS, vs = g % C::kVS;
+          if (!(ok = mbar_wait(B.pk_full + s, (g / C::kPS) & 1, abort_flag))) break;
+          if (!(ok = mbar_wait(B.kw_empty + ks, ((g / C::kKS) & 1) ^ 1, abort_flag))) break;
+          const uint8_t* pk = smem + C::oPk + s * 2 * C::kPkHalf;
+          widen_tile<D>(pk, smem + C::oKw + ks * C::kKwStride, BN, wt, 64);
+          if (wt < BN) {
+            const int j = t * BN + wt;
+            float* ksc = reinterpret_cast<float*>(smem + C::oKsc) + ks * BN;
+            ksc[wt] = j < prm.N ? prm.sk[static_cast<size_t>(bh) * prm.N + j] * (1.0f / 256.0f) : 0.0f;
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(B.kw_full + ks);
+          if (!(ok = mbar_wait(B.vw_empty + vs, ((g / C::kVS) & 1) ^ 1, abort_flag))) break;
+          widen_tile<D>(pk + C::kPkHalf, smem + C::oVw + vs * C::kVwStride, BN, wt, 64);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) { mbar_arrive(B.vw_full + vs); mbar_arrive(B.pk_empty + s); }
+        }
+      }
+      if (!ok) set_status(kStatusTimeout);
+    }
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 232;");
+    // -------------------------------------------------------------- softmax
+    const int tt = (warp - 4) >> 2;               // query tile of this warpgroup
+    const int quad = warp & 3;                    // TMEM lane quadrant
+    const int r = quad * 32 + lane;               // row within the tile
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const uint32_t tA = tbase + tt * 256 + 128 + lane_off;
+    const float kLog2e = 1.4426950408889634f;
+    uint32_t g = 0;
+    bool ok = true;
+    float F[D];
+    for (int item = blockIdx.x; item < prm.nitems && ok; item += gridDim.x) {
+      const int bh = item / prm.npairs, pair = item % prm.npairs;
+      const int qtile = pair * 2 + tt;
+      const int row = qtile * kRows + r;
+      const bool row_ok = row < prm.N;
+      const float ci = row_ok ? __fmul_rn(prm.sq[static_cast<size_t>(bh) * prm.N + row], prm.inv_sqrt_d) : 0.0f;
+      const float cpi = __fmul_rn(ci, kLog2e);
+      const bool dump_tile = DUMP && bh == prm.dump_bh && qtile == prm.dump_tile && row_ok;
+#pragma unroll
+      for (int i = 0; i < D; ++i) F[i] = 0.0f;
+      float m_run = -INFINITY, m_ref = 0.0f, w = 1.0f, Lf = 0.0f;
+      int Lrun = 0;
+      // fresh integer accumulator
+#pragma unroll
+      for (int c = 0; c < D; c += 32) tmem_fill32(tA + c, kMagic);
+      for (int t = 0; t < nb; ++t, ++g) {
+        const uint32_t buf = g & 1;
+        const uint32_t tS = tbase + tt * 256 + buf * 64 + lane_off;
+        if (!(ok = mbar_wait(B.s_full + tt * 2 + buf, (g >> 1) & 1, abort_flag))) break;
+        tc_fence_after();
+        uint32_t raw[BN];
+        tmem_ld<BN>(tS, raw);
+        const int ks = g % C::kKS;
+        if (!(ok = mbar_wait(B.kw_full + ks, (g / C::kKS) & 1, abort_flag))) break;
+        const float* ksc = reinterpret_cast<const float*>(smem + C::oKsc) + ks * BN;
+        tmem_wait_ld();
+        const int nvalid = min(BN, prm.N - t * BN);
+        float v[BN];
+#pragma unroll
+        for (int j = 0; j < BN; ++j) {
+          const float f = __int_as_float(static_cast<int>(raw[j]) + static_cast<int>(kMagic)) - kMagicF;
+          v[j] = f * ksc[j];
+        }
+        if (nvalid < BN) {
+#pragma unroll
+          for (int j = 0; j < BN; ++j)
+            if (j >= nvalid) v[j] = -INFINITY;
+        }
+        float vmax = v[0];
+#pragma unroll
+        for (int j = 1; j + 1 < BN; j += 2) vmax = max3(vmax, v[j], v[j + 1]);
+        if (BN % 2 == 0) vmax = fmaxf(vmax, v[BN - 1]);
+        const float m_blk = __fmul_rn(vmax, ci);
+        const float m_new = fmaxf(m_run, m_blk);
+        const bool grow = m_new > m_run;
+        const float Mp = __fmul_rn(m_new, kLog2e);
+        uint32_t words[C::kKeysPV / 4];
+        int lq = 0;
+#pragma unroll
+        for (int q = 0; q < BN / 4; ++q) {
+          uint32_t tb[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int j = 4 * q + e;
+            float y = fmaf(v[j], cpi, -Mp);
+            if (nvalid < BN && j >= nvalid) y = -INFINITY;
+            const float pe = ex2_approx(y);
+            tb[e] = __float_as_uint(fmaf(15.0f, pe, kMagicF));
+          }
+          const uint32_t wd = __byte_perm(__byte_perm(tb[0], tb[1], 0x0040), __byte_perm(tb[2], tb[3], 0x0040), 0x5410);
+          words[q] = wd;
+          lq = __dp4a(static_cast<int>(wd), 0x01010101, lq);
+        }
+#pragma unroll
+        for (int q = BN / 4; q < C::kKeysPV / 4; ++q) words[q] = 0u;
+        if constexpr (C::kKeysPV / 4 == 16) tmem_st16(tS, words);
+        else if constexpr (C::kKeysPV / 4 == 8) tmem_st8(tS, words);
+        if (dump_tile) {
+          for (int j = 0; j < nvalid; ++j) {
+            const size_t o = static_cast<size_t>(r) * prm.N + t * BN + j;
+            if (prm.dump_s) prm.dump_s[o] = static_cast<int32_t>(raw[j]) / 256;
+            if (prm.dump_p) prm.dump_p[o] = static_cast<int8_t>(((words[j >> 2] >> (8 * (j & 3))) & 0xFF) - 8);
+          }
+        }
+        // Fold the integer accumulator into F when a row's maximum grows (its
+        // earlier codes used the old maximum) or its magnitude bound is near
+        // the exact range of the read-back (|acc| < 2^22).
+        const bool near_bound = (Lrun + 15 * BN) * 112 >= (1 << 22) - 4096;
+        const bool need = (t > 0) && (grow || near_bound || DUMP);
+        if (__any_sync(0xFFFFFFFFu, need)) {
+          if (!(ok = mbar_wait(B.pv_done + tt, (g - 1) & 1, abort_flag))) break;
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < D; c += 32) {
+            uint32_t a[32];
+            tmem_ld32(tA + c, a);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float af = __int_as_float(static_cast<int>(a[i])) - kMagicF;
+              F[c + i] = fmaf(w, af, F[c + i]);
+              if (dump_tile && prm.dump_acc)
+                prm.dump_acc[(static_cast<size_t>(r) * nb + (t - 1)) * D + wide_to_dim(c + i)] =
+                    (static_cast<int>(a[i]) - static_cast<int>(kMagic)) / 16;
+            }
+            tmem_fill32(tA + c, kMagic);
+          }
+          Lf = fmaf(w, static_cast<float>(Lrun), Lf);
+          Lrun = 0;
+        }
+        if (t == 0) {
+          m_ref = m_new;
+          w = 1.0f;
+        } else if (grow) {
+          const float x = __fmul_rn(m_new - m_ref, kLog2e);
+          if (x > 64.0f) {
+            const float sc = ex2_approx(-x);
+#pragma unroll
+            for (int i = 0; i < D; ++i) F[i] *= sc;
+            Lf *= sc;
+            m_ref = m_new;
+            w = 1.0f;
+          } else {
+            w = ex2_approx(x);
+          }
+        }
+        Lrun += lq;
+        m_run = m_new;
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(B.p_full + tt * 2 + buf);
+          mbar_arrive(B.kw_empty + ks);
+        }
+      }
+      if (!ok) break;
+      // Last block: fold the accumulator, normalise, store.
+      if (!(ok = mbar_wait(B.pv_done + tt, (g - 1) & 1, abort_flag))) break;
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < D; c += 32) {
+        uint32_t a[32];
+        tmem_ld32(tA + c, a);
+        tmem_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const float af = __int_as_float(static_cast<int>(a[i])) - kMagicF;
+          F[c + i] = fmaf(w, af, F[c + i]);
+          if (dump_tile && prm.dump_acc)
+            prm.dump_acc[(static_cast<size_t>(r) * nb + (nb - 1)) * D + wide_to_dim(c + i)] =
+                (static_cast<int>(a[i]) - static_cast<int>(kMagic)) / 16;
+        }
+      }
+      Lf = fmaf(w, static_cast<float>(Lrun), Lf);
+      if (row_ok) {
+        const float inv = 1.0f / (16.0f * Lf);
+        const float* sv = prm.sv + static_cast<size_t>(bh) * D;
+        __nv_bfloat16* orow = prm.out + (static_cast<size_t>(bh) * prm.N + row) * D;
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+              const int d = c + 8 * a + 2 * b;
+              const float o0 = F[c + 4 * a + b] * __ldg(sv + d) * inv;
+              const float o1 = F[c + 16 + 4 * a + b] * __ldg(sv + d + 1) * inv;
+              const __nv_bfloat162 h = __floats2bfloat162_rn(o0, o1);
+              pk[4 * a + b] = *reinterpret_cast<const uint32_t*>(&h);
+            }
+          uint4* dst = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+          for (int u = 0; u < 4; ++u) dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+        }
+        if (prm.lse) prm.lse[static_cast<size_t>(bh) * prm.N + row] = m_ref + logf(Lf * (1.0f / 15.0f));
+      }
+    }
+    if (!ok) set_status(kStatusTimeout);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tbase, 512);
+}
+
+// ------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 get_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 3D map over packed codes [BH, N, D/2] bytes; box = rows x D/2; zero fill past N.
+bool make_code_map(CUtensorMap* m, const void* base, int BH, int N, int D, int rows) {
+  auto enc = get_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D / 2), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D / 2), static_cast<cuuint64_t>(N) * (D / 2)};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(D / 2), static_cast<cuuint32_t>(rows), 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D, int BN, bool DUMP>
+cudaError_t launch_cfg(const ra_problem& p, const uint8_t* q4, const uint8_t* k4, const uint8_t* v4,
+                       const AttnParams& prm, cudaStream_t st) {
+  using C = Cfg<D, BN>;
+  CUtensorMap mq, mk, mv;
+  const int BH = p.B * p.H;
+  if (!make_code_map(&mq, q4, BH, p.N, D, kRows) || !make_code_map(&mk, k4, BH, p.N, D, BN) ||
+      !make_code_map(&mv, v4, BH, p.N, D, BN))
+    return cudaErrorInvalidValue;
+  auto kern = attn_int4_kernel<D, BN, DUMP>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, nsm = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = prm.nitems < nsm ? prm.nitems : nsm;
+  kern<<<grid, kThreads, C::kSmem, st>>>(mq, mk, mv, prm);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attn_int4(const ra_problem& p, const uint8_t* q4, const float* sq, const uint8_t* k4,
+                             const float* sk, const uint8_t* v4, const float* sv, void* out, float* lse,
+                             const AttnDump* dump, cudaStream_t st, int* unsupported) {
+  AttnParams prm{};
+  prm.N = p.N;
+  prm.BH = p.B * p.H;
+  prm.nblocks = (p.N + p.block_k - 1) / p.block_k;
+  prm.npairs = (p.N + 2 * kRows - 1) / (2 * kRows);
+  prm.nitems = prm.BH * prm.npairs;
+  prm.inv_sqrt_d = static_cast<float>(1.0 / sqrt(static_cast<double>(p.D)));
+  prm.sq = sq; prm.sk = sk; prm.sv = sv;
+  prm.out = static_cast<__nv_bfloat16*>(out);
+  prm.lse = lse;
+  const bool dmp = dump != nullptr;
+  if (dmp) {
+    prm.dump_bh = dump->bh; prm.dump_tile = dump->q_tile;
+    prm.dump_s = dump->s; prm.dump_p = dump->p; prm.dump_acc = dump->acc;
+  }
+  *unsupported = 0;
+#define RA_CASE(DD, BB)                                                                              \
+  if (p.D == DD && p.block_k == BB)                                                                  \
+    return dmp ? launch_cfg<DD, BB, true>(p, q4, k4, v4, prm, st) : launch_cfg<DD, BB, false>(p, q4, k4, v4, prm, st);
+  RA_CASE(128, 64)
+  RA_CASE(128, 32)
+  RA_CASE(128, 16)
+  RA_CASE(64, 64)
+  RA_CASE(64, 32)
+  RA_CASE(64, 16)
+#undef RA_CASE
+  *unsupported = 1;
+  return cudaSuccess;
+}
+
+cudaError_t read_attn_int4_status(uint32_t* out) {
+  uint32_t zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(out, g_attn_status, sizeof(uint32_t));
+  if (e != cudaSuccess) return e;
+  return cudaMemcpyToSymbol(g_attn_status, &zero, sizeof(uint32_t));
+}
+
+}  // namespace ra

@@ -1,0 +1,449 @@
+// Fused prologue of the RotateAttention INT4 forward (memory-bound):
+//   3D RoPE + RoPE-aware rotation of Q and K, K smoothing, per-token INT4 of Q
+//   and K, per-channel INT4 of V and per-block V column sums; plus the plain
+//   RoPE to bf16 that feeds the bf16 fallback.
+// Method: RotateAttention (arXiv 2607.02584), papernotes page "overall
+// framework" and "key design 1"; gecl notes "Key Insight" (per-token INT4).
+//
+// Every value that decides a code is computed in fp32 with explicit
+// round-to-nearest intrinsics in a fixed order (no contraction), so codes
+// match an fp32 reference of the same definition bit for bit.
+//
+// Layout: 8 consecutive channels per thread, D/8 threads per token, so a warp
+// reads 512 contiguous bytes of bf16 per token pair with 16-byte loads.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "ra_common.cuh"
+#include "ra_internal.h"
+
+namespace ra {
+namespace {
+
+__device__ uint32_t g_prologue_status = 0;
+
+constexpr int kThreads = 256;
+constexpr int kChunk = 256;  // tokens per CTA; a multiple of every block_k
+
+struct SegInfo {
+  int off[3];     // first channel of each segment
+  int dj[3];      // channels of each segment
+  int toff[3];    // first table entry of each segment
+  int grid[3];
+};
+
+__device__ __forceinline__ void load8(const void* base, size_t elem_off, int dtype, float* x) {
+  if (dtype == 1) {
+    const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(base) + elem_off);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      x[2 * i] = __uint_as_float(w[i] << 16);
+      x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  } else {
+    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(base) + elem_off);
+    const float4 a = p[0], b = p[1];
+    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+  }
+}
+
+__device__ __forceinline__ int seg_of(const SegInfo& s, int d) {
+  return d < s.off[1] ? 0 : (d < s.off[2] ? 1 : 2);
+}
+
+// Reads the token's grid position; a position outside the grid is reported and
+// clamped so every table access stays in bounds.
+__device__ __forceinline__ int grid_pos(const SegInfo& s, const int32_t* pos, int n, int j) {
+  int g = pos[3 * n + j];
+  if (g < 0 || g >= s.grid[j]) {
+    atomicOr(&g_prologue_status, kStatusBadPosition);
+    g = g < 0 ? 0 : s.grid[j] - 1;
+  }
+  return g;
+}
+
+// RoPE (+ rotation) of this thread's 8 channels [c0, c0+8) of token n.
+//   rot 1 (interleaved, fused table): y0 = x0 a + x1 b, y1 = x0 b - x1 a
+//   rot 0 / 2: y0 = x0 c - x1 s, y1 = x0 s + x1 c; rot 2 then pairs i, i + Dj/2
+//   through the per-warp row buffer `row` (D floats for this token).
+__device__ __forceinline__ void rope_rotate8(const SegInfo& s, const float* tab_a, const float* tab_b,
+                                             const int32_t* pos, int n, int rot, int c0, float* x,
+                                             float* row) {
+#pragma unroll
+  for (int pr = 0; pr < 4; ++pr) {
+    const int d = c0 + 2 * pr;
+    const int j = seg_of(s, d);
+    const int k = (d - s.off[j]) >> 1;
+    const int g = grid_pos(s, pos, n, j);
+    const int idx = s.toff[j] + g * (s.dj[j] >> 1) + k;
+    const float a = __ldg(tab_a + idx), b = __ldg(tab_b + idx);
+    const float x0 = x[2 * pr], x1 = x[2 * pr + 1];
+    if (rot == 1) {
+      x[2 * pr] = __fadd_rn(__fmul_rn(x0, a), __fmul_rn(x1, b));
+      x[2 * pr + 1] = __fsub_rn(__fmul_rn(x0, b), __fmul_rn(x1, a));
+    } else {
+      x[2 * pr] = __fsub_rn(__fmul_rn(x0, a), __fmul_rn(x1, b));
+      x[2 * pr + 1] = __fadd_rn(__fmul_rn(x0, b), __fmul_rn(x1, a));
+    }
+  }
+  if (rot == 2) {
+    const float r2 = 0.70710678118654752440f;  // fp32 rounding of 1/sqrt(2)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) row[c0 + i] = x[i];
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int d = c0 + i;
+      const int j = seg_of(s, d);
+      const int h = s.dj[j] >> 1;
+      const int t = (d - s.off[j]) >> 1;
+      const float u = row[s.off[j] + t], w = row[s.off[j] + t + h];
+      x[i] = (d - s.off[j]) & 1 ? __fmul_rn(__fsub_rn(u, w), r2) : __fmul_rn(__fadd_rn(u, w), r2);
+    }
+    __syncwarp();
+  }
+}
+
+// rint(y) for |y| < 2^22 with ties to even: adding 1.5 * 2^23 rounds to an integer.
+__device__ __forceinline__ int rint_small(float y) {
+  return __float_as_int(__fadd_rn(y, 12582912.0f)) - 0x4B400000;
+}
+
+__device__ __forceinline__ int quant4(float x, float inv) {
+  int c = rint_small(__fmul_rn(x, inv));
+  return c > 7 ? 7 : (c < -7 ? -7 : c);
+}
+
+__device__ __forceinline__ uint32_t pack8(const int* c) {
+  uint32_t w = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) w |= static_cast<uint32_t>(c[i] & 0xF) << (4 * i);
+  return w;
+}
+
+// Max over the D/8 threads of a token (a contiguous lane group of size lpt).
+__device__ __forceinline__ float group_max(float v, int lpt) {
+  for (int o = lpt >> 1; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
+}
+
+struct PrologueArgs {
+  SegInfo s;
+  int N, D, rot, dtype, block_k, nchunk;
+  const void *q, *k, *v;
+  const int32_t* pos;
+  const float *tab_a, *tab_b;
+  double* ksum;     // [BH, nchunk, D]
+  float* vmax;      // [BH, nchunk, D]
+  float* vinv;      // [BH, D]
+  uint8_t *q4, *k4, *v4;
+  float *sq, *sk, *k_mean, *sv;
+  int32_t* colsum;
+};
+
+// Table entry e -> (segment j, position g, pair k); angle g * theta^(-2k/Dj) in
+// fp64, entries rounded once to fp32.  rot 1 stores the fused H2 block.
+__global__ void rope_table_kernel(SegInfo s, int total, double theta, int rot, float* tab_a, float* tab_b) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= total) return;
+  const int j = e < s.toff[1] ? 0 : (e < s.toff[2] ? 1 : 2);
+  const int npair = s.dj[j] >> 1;
+  const int g = (e - s.toff[j]) / npair, k = (e - s.toff[j]) % npair;
+  const double freq = pow(theta, -2.0 * static_cast<double>(k) / static_cast<double>(s.dj[j]));
+  const double phi = static_cast<double>(g) * freq;
+  const double c = cos(phi), sn = sin(phi);
+  if (rot == 1) {
+    tab_a[e] = static_cast<float>((c + sn) / sqrt(2.0));
+    tab_b[e] = static_cast<float>((c - sn) / sqrt(2.0));
+  } else {
+    tab_a[e] = static_cast<float>(c);
+    tab_b[e] = static_cast<float>(sn);
+  }
+}
+
+// Pass 1: per chunk of tokens, fp64 channel sums of the rotated K and channel
+// maxima of |V|.
+__global__ void __launch_bounds__(kThreads) prologue_reduce_kernel(PrologueArgs a) {
+  __shared__ float rows[kThreads / 32][4][128];
+  __shared__ double red_s[kThreads][8];
+  __shared__ float red_m[kThreads][8];
+  const int bh = blockIdx.y, chunk = blockIdx.x;
+  const int lpt = a.D >> 3, tpw = 32 / lpt;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tok_in_warp = lane / lpt, c0 = (lane % lpt) * 8;
+  double ks[8];
+  float vm[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) { ks[i] = 0.0; vm[i] = 0.0f; }
+  const int n0 = chunk * kChunk;
+  const size_t head = static_cast<size_t>(bh) * a.N * a.D;
+  for (int base = n0; base < n0 + kChunk; base += (kThreads / 32) * tpw) {
+    const int n = base + warp * tpw + tok_in_warp;
+    const bool ok = n < a.N;
+    float x[8], y[8];
+    if (ok) {
+      load8(a.k, head + static_cast<size_t>(n) * a.D + c0, a.dtype, x);
+      load8(a.v, head + static_cast<size_t>(n) * a.D + c0, a.dtype, y);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) { x[i] = 0.0f; y[i] = 0.0f; }
+    }
+    // rope_rotate8 synchronises the warp for the half rotation, so every lane
+    // takes part; lanes past N carry zeros and position 0.
+    rope_rotate8(a.s, a.tab_a, a.tab_b, a.pos, ok ? n : 0, a.rot, c0, x, rows[warp][tok_in_warp]);
+    if (ok) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        ks[i] += static_cast<double>(x[i]);
+        vm[i] = fmaxf(vm[i], fabsf(y[i]));
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) { red_s[threadIdx.x][i] = ks[i]; red_m[threadIdx.x][i] = vm[i]; }
+  __syncthreads();
+  // Threads t with t % lpt == c hold channels [8c, 8c+8); fold them in thread order.
+  for (int d = threadIdx.x; d < a.D; d += kThreads) {
+    const int c = d >> 3, i = d & 7;
+    double sum = 0.0;
+    float mx = 0.0f;
+    for (int t = c; t < kThreads; t += lpt) {
+      sum += red_s[t][i];
+      mx = fmaxf(mx, red_m[t][i]);
+    }
+    const size_t o = (static_cast<size_t>(bh) * a.nchunk + chunk) * a.D + d;
+    a.ksum[o] = sum;
+    a.vmax[o] = mx;
+  }
+}
+
+// Per head and channel: K mean (fp64 sum over chunks in order, rounded once),
+// V scale amax/7 and reciprocal 7/amax.
+__global__ void prologue_finalize_kernel(PrologueArgs a) {
+  const int bh = blockIdx.x, d = threadIdx.x;
+  if (d >= a.D) return;
+  double sum = 0.0;
+  float mx = 0.0f;
+  for (int c = 0; c < a.nchunk; ++c) {
+    const size_t o = (static_cast<size_t>(bh) * a.nchunk + c) * a.D + d;
+    sum += a.ksum[o];
+    mx = fmaxf(mx, a.vmax[o]);
+  }
+  a.k_mean[bh * a.D + d] = static_cast<float>(sum / static_cast<double>(a.N));
+  a.sv[bh * a.D + d] = __fdiv_rn(mx, 7.0f);
+  a.vinv[bh * a.D + d] = mx == 0.0f ? 0.0f : __fdiv_rn(7.0f, mx);
+}
+
+// Pass 2: quantise.  Q, K: rotate (K also smoothed), per-token scale and codes.
+// V: per-channel codes, column sums per key block.
+__global__ void __launch_bounds__(kThreads) prologue_quant_kernel(PrologueArgs a) {
+  __shared__ float rows[kThreads / 32][4][128];
+  __shared__ int csum[kChunk / 16][128];
+  const int bh = blockIdx.y, chunk = blockIdx.x;
+  const int lpt = a.D >> 3, tpw = 32 / lpt;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tok_in_warp = lane / lpt, c0 = (lane % lpt) * 8;
+  const int nblk = kChunk / a.block_k;
+  for (int i = threadIdx.x; i < nblk * a.D; i += kThreads) csum[i / a.D][i % a.D] = 0;
+  float kmean[8], vinv[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    kmean[i] = a.k_mean[bh * a.D + c0 + i];
+    vinv[i] = a.vinv[bh * a.D + c0 + i];
+  }
+  __syncthreads();
+  const int n0 = chunk * kChunk;
+  const size_t head = static_cast<size_t>(bh) * a.N * a.D;
+  const size_t head4 = static_cast<size_t>(bh) * a.N * (a.D / 2);
+  for (int base = n0; base < n0 + kChunk; base += (kThreads / 32) * tpw) {
+    const int n = base + warp * tpw + tok_in_warp;
+    const bool ok = n < a.N;
+    const int nn = ok ? n : 0;
+    float xq[8], xk[8], xv[8];
+    if (ok) {
+      load8(a.q, head + static_cast<size_t>(n) * a.D + c0, a.dtype, xq);
+      load8(a.k, head + static_cast<size_t>(n) * a.D + c0, a.dtype, xk);
+      load8(a.v, head + static_cast<size_t>(n) * a.D + c0, a.dtype, xv);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) { xq[i] = 0.0f; xk[i] = 0.0f; xv[i] = 0.0f; }
+    }
+    rope_rotate8(a.s, a.tab_a, a.tab_b, a.pos, nn, a.rot, c0, xq, rows[warp][tok_in_warp]);
+    rope_rotate8(a.s, a.tab_a, a.tab_b, a.pos, nn, a.rot, c0, xk, rows[warp][tok_in_warp]);
+    float mq = 0.0f, mk = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      xk[i] = __fsub_rn(xk[i], kmean[i]);
+      mq = fmaxf(mq, fabsf(xq[i]));
+      mk = fmaxf(mk, fabsf(xk[i]));
+    }
+    mq = group_max(mq, lpt);
+    mk = group_max(mk, lpt);
+    int cq[8], ck[8], cv[8];
+    const float iq = mq == 0.0f ? 0.0f : __fdiv_rn(7.0f, mq);
+    const float ik = mk == 0.0f ? 0.0f : __fdiv_rn(7.0f, mk);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      cq[i] = quant4(xq[i], iq);
+      ck[i] = quant4(xk[i], ik);
+      cv[i] = quant4(xv[i], vinv[i]);
+    }
+    if (ok) {
+      const size_t o4 = head4 + static_cast<size_t>(n) * (a.D / 2) + (c0 >> 1);
+      *reinterpret_cast<uint32_t*>(a.q4 + o4) = pack8(cq);
+      *reinterpret_cast<uint32_t*>(a.k4 + o4) = pack8(ck);
+      *reinterpret_cast<uint32_t*>(a.v4 + o4) = pack8(cv);
+      if (c0 == 0) {
+        a.sq[static_cast<size_t>(bh) * a.N + n] = __fdiv_rn(mq, 7.0f);
+        a.sk[static_cast<size_t>(bh) * a.N + n] = __fdiv_rn(mk, 7.0f);
+      }
+      const int blk = (n - n0) / a.block_k;
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (cv[i] != 0) atomicAdd(&csum[blk][c0 + i], cv[i]);
+    }
+  }
+  __syncthreads();
+  const int nb_total = (a.N + a.block_k - 1) / a.block_k;
+  for (int i = threadIdx.x; i < nblk * a.D; i += kThreads) {
+    const int bl = i / a.D, d = i % a.D;
+    const int gb = chunk * nblk + bl;
+    if (gb < nb_total) a.colsum[(static_cast<size_t>(bh) * nb_total + gb) * a.D + d] = csum[bl][d];
+  }
+}
+
+// RoPE only (rotation off) to bf16, round to nearest even.
+__global__ void __launch_bounds__(kThreads) rope_bf16_kernel(PrologueArgs a, __nv_bfloat16* qo,
+                                                             __nv_bfloat16* ko) {
+  __shared__ float rows[kThreads / 32][4][128];
+  const int bh = blockIdx.y, chunk = blockIdx.x;
+  const int lpt = a.D >> 3, tpw = 32 / lpt;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tok_in_warp = lane / lpt, c0 = (lane % lpt) * 8;
+  const int n0 = chunk * kChunk;
+  const size_t head = static_cast<size_t>(bh) * a.N * a.D;
+  for (int base = n0; base < n0 + kChunk; base += (kThreads / 32) * tpw) {
+    const int n = base + warp * tpw + tok_in_warp;
+    if (n >= a.N) continue;
+    float x[8];
+#pragma unroll
+    for (int which = 0; which < 2; ++which) {
+      load8(which ? a.k : a.q, head + static_cast<size_t>(n) * a.D + c0, a.dtype, x);
+      rope_rotate8(a.s, a.tab_a, a.tab_b, a.pos, n, 0, c0, x, rows[warp][tok_in_warp]);
+      uint32_t w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 h2 = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+        w[i] = *reinterpret_cast<const uint32_t*>(&h2);
+      }
+      __nv_bfloat16* dst = (which ? ko : qo) + head + static_cast<size_t>(n) * a.D + c0;
+      *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+}
+
+SegInfo seg_info(const ra_problem& p) {
+  SegInfo s;
+  int o = 0, t = 0;
+  for (int j = 0; j < 3; ++j) {
+    s.off[j] = o;
+    s.dj[j] = p.seg[j];
+    s.toff[j] = t;
+    s.grid[j] = p.grid[j];
+    o += p.seg[j];
+    t += p.grid[j] * (p.seg[j] / 2);
+  }
+  return s;
+}
+
+}  // namespace
+
+size_t rope_table_len(const ra_problem& p) {
+  size_t t = 0;
+  for (int j = 0; j < 3; ++j) t += static_cast<size_t>(p.grid[j]) * (p.seg[j] / 2);
+  return t;
+}
+
+int prologue_nchunk(const ra_problem& p) { return (p.N + kChunk - 1) / kChunk; }
+
+static size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+WorkspaceLayout workspace_layout(const ra_problem& p) {
+  WorkspaceLayout w;
+  const size_t bh = static_cast<size_t>(p.B) * p.H, T = rope_table_len(p), nc = prologue_nchunk(p);
+  size_t o = 0;
+  w.tab_a = o; o = align256(o + T * sizeof(float));
+  w.tab_b = o; o = align256(o + T * sizeof(float));
+  w.ksum = o;  o = align256(o + bh * nc * p.D * sizeof(double));
+  w.vmax = o;  o = align256(o + bh * nc * p.D * sizeof(float));
+  w.vinv = o;  o = align256(o + bh * p.D * sizeof(float));
+  w.total = o;
+  return w;
+}
+
+static cudaError_t launch_tables(const ra_problem& p, int rot, float* ta, float* tb, cudaStream_t st) {
+  const SegInfo s = seg_info(p);
+  const int T = static_cast<int>(rope_table_len(p));
+  rope_table_kernel<<<(T + 255) / 256, 256, 0, st>>>(s, T, static_cast<double>(p.theta), rot, ta, tb);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prologue(const ra_problem& p, int dtype, const void* q, const void* k, const void* v,
+                            const int32_t* pos, uint8_t* q4, float* sq, uint8_t* k4, float* sk,
+                            float* k_mean, uint8_t* v4, float* sv, int32_t* colsum, void* ws,
+                            cudaStream_t st) {
+  const WorkspaceLayout w = workspace_layout(p);
+  char* base = static_cast<char*>(ws);
+  PrologueArgs a;
+  a.s = seg_info(p);
+  a.N = p.N; a.D = p.D; a.rot = p.rot; a.dtype = dtype; a.block_k = p.block_k;
+  a.nchunk = prologue_nchunk(p);
+  a.q = q; a.k = k; a.v = v; a.pos = pos;
+  a.tab_a = reinterpret_cast<float*>(base + w.tab_a);
+  a.tab_b = reinterpret_cast<float*>(base + w.tab_b);
+  a.ksum = reinterpret_cast<double*>(base + w.ksum);
+  a.vmax = reinterpret_cast<float*>(base + w.vmax);
+  a.vinv = reinterpret_cast<float*>(base + w.vinv);
+  a.q4 = q4; a.k4 = k4; a.v4 = v4; a.sq = sq; a.sk = sk; a.k_mean = k_mean; a.sv = sv;
+  a.colsum = colsum;
+  cudaError_t e = launch_tables(p, p.rot, const_cast<float*>(a.tab_a), const_cast<float*>(a.tab_b), st);
+  if (e != cudaSuccess) return e;
+  const dim3 grid(a.nchunk, p.B * p.H);
+  prologue_reduce_kernel<<<grid, kThreads, 0, st>>>(a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  prologue_finalize_kernel<<<p.B * p.H, 128, 0, st>>>(a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  prologue_quant_kernel<<<grid, kThreads, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rope_bf16(const ra_problem& p, int dtype, const void* q, const void* k,
+                             const int32_t* pos, void* qo, void* ko, void* ws, cudaStream_t st) {
+  const WorkspaceLayout w = workspace_layout(p);
+  char* base = static_cast<char*>(ws);
+  PrologueArgs a{};
+  a.s = seg_info(p);
+  a.N = p.N; a.D = p.D; a.rot = 0; a.dtype = dtype; a.block_k = p.block_k;
+  a.nchunk = prologue_nchunk(p);
+  a.q = q; a.k = k; a.pos = pos;
+  a.tab_a = reinterpret_cast<float*>(base + w.tab_a);
+  a.tab_b = reinterpret_cast<float*>(base + w.tab_b);
+  cudaError_t e = launch_tables(p, 0, const_cast<float*>(a.tab_a), const_cast<float*>(a.tab_b), st);
+  if (e != cudaSuccess) return e;
+  rope_bf16_kernel<<<dim3(a.nchunk, p.B * p.H), kThreads, 0, st>>>(a, static_cast<__nv_bfloat16*>(qo),
+                                                                   static_cast<__nv_bfloat16*>(ko));
+  return cudaGetLastError();
+}
+
+cudaError_t read_prologue_status(uint32_t* out) {
+  uint32_t zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(out, g_prologue_status, sizeof(uint32_t));
+  if (e != cudaSuccess) return e;
+  return cudaMemcpyToSymbol(g_prologue_status, &zero, sizeof(uint32_t));
+}
+
+}  // namespace ra

@@ -35,6 +35,7 @@ def lib():
         _lib.orc_prologue_head.argtypes = [P(OrcProblem)] + [vp] * 14
         _lib.orc_p_code.argtypes = [C.c_float, C.c_float]
         _lib.orc_attention_int4_rows.argtypes = [P(OrcProblem)] + [vp] * 7 + [C.c_int, C.c_int] + [vp] * 5
+        _lib.orc_attention_int4_rows_given_codes.argtypes = [P(OrcProblem)] + [vp] * 8 + [C.c_int, C.c_int, vp, vp]
         _lib.orc_attention_exact_blocked_rows.argtypes = [P(OrcProblem), vp, vp, vp, C.c_int, C.c_int, vp, vp]
         _lib.orc_rotation_matrix.argtypes = [P(OrcProblem), vp]
         _lib.orc_rope_matrix.argtypes = [P(OrcProblem), vp, vp]
@@ -139,6 +140,21 @@ def attention_int4_rows(p: OrcProblem, h: Dict[str, np.ndarray], row0: int, row1
                                        _ptr(r.get("codes")), _ptr(r.get("acc")))
     _check(rc, "attention_int4_rows")
     return r
+
+
+def attention_int4_rows_given_codes(p: OrcProblem, h: Dict[str, np.ndarray], codes: np.ndarray,
+                                    row0: int, row1: int) -> Dict[str, np.ndarray]:
+    """INT4 attention of rows [row0, row1) with the P codes given ([rows, N] int8)."""
+    R = row1 - row0
+    out = np.empty((R, p.D), np.float64)
+    lse = np.empty(R, np.float64)
+    codes = np.ascontiguousarray(codes, np.int8)
+    assert codes.shape == (R, p.N)
+    args = [np.ascontiguousarray(h[k]) for k in ("q4", "sq", "k4", "sk", "v4", "sv", "colsum")]
+    rc = lib().orc_attention_int4_rows_given_codes(C.byref(p), *[_ptr(a) for a in args], _ptr(codes),
+                                                   int(row0), int(row1), _ptr(out), _ptr(lse))
+    _check(rc, "attention_int4_rows_given_codes")
+    return {"out": out, "lse": lse}
 
 
 def attention_exact_blocked_rows(p: OrcProblem, q: np.ndarray, k: np.ndarray, v: np.ndarray,

@@ -345,6 +345,8 @@ typedef struct {
   const float *sq, *sk, *sv;
   const int32_t* colsum;
   const double *qf, *kf, *vf;
+  const int8_t* codes_in;  /* nullable [rows, N]: P codes to use instead of computing them */
+  int row0;
 } orc_attn_in;
 
 static void attn_row(const orc_problem* p, const orc_attn_in* in, int quant, int i,
@@ -387,7 +389,7 @@ static void attn_row(const orc_problem* p, const orc_attn_in* in, int quant, int
       int32_t acci[256];
       for (int d = 0; d < D; ++d) acci[d] = 0;
       for (int j = j0; j < j1; ++j) {
-        int c = orc_p_code(S[j - j0], m);
+        int c = in->codes_in ? in->codes_in[(size_t)(i - in->row0) * N + j] : orc_p_code(S[j - j0], m);
         if (c_dump) c_dump[j] = (int8_t)c;
         lq += c + 8;
         const uint8_t* vr = in->v4 + (size_t)j * (D / 2);
@@ -446,8 +448,26 @@ int orc_attention_int4_rows(const orc_problem* p, const uint8_t* q4, const float
                             double* out, double* lse, int32_t* s_dump, int8_t* c_dump,
                             int32_t* acc_dump) {
   if (check_problem(p) || row0 < 0 || row1 > p->N || row0 >= row1) return ORC_BAD;
-  orc_attn_in in = {q4, k4, v4, sq, sk, sv, colsum, NULL, NULL, NULL};
+  orc_attn_in in = {q4, k4, v4, sq, sk, sv, colsum, NULL, NULL, NULL, NULL, row0};
   attn_rows(p, &in, 1, row0, row1, out, lse, s_dump, c_dump, acc_dump);
+  return ORC_OK;
+}
+
+/*
+ * The same INT4 attention with the P codes supplied by the caller
+ * (codes_in [row1-row0, N], values in [-8, 7]) instead of computed: the
+ * running maximum, the online rescaling and the accumulation are unchanged.
+ * Used to check an implementation's accumulation on its own codes.
+ */
+int orc_attention_int4_rows_given_codes(const orc_problem* p, const uint8_t* q4, const float* sq,
+                                        const uint8_t* k4, const float* sk, const uint8_t* v4,
+                                        const float* sv, const int32_t* colsum, const int8_t* codes_in,
+                                        int row0, int row1, double* out, double* lse) {
+  if (check_problem(p) || row0 < 0 || row1 > p->N || row0 >= row1 || !codes_in) return ORC_BAD;
+  for (size_t i = 0; i < (size_t)(row1 - row0) * p->N; ++i)
+    if (codes_in[i] < -8 || codes_in[i] > 7) return ORC_BAD;
+  orc_attn_in in = {q4, k4, v4, sq, sk, sv, colsum, NULL, NULL, NULL, codes_in, row0};
+  attn_rows(p, &in, 1, row0, row1, out, lse, NULL, NULL, NULL);
   return ORC_OK;
 }
 
@@ -455,7 +475,7 @@ int orc_attention_exact_blocked_rows(const orc_problem* p, const double* q, cons
                                      const double* v, int row0, int row1, double* out,
                                      double* lse) {
   if (check_problem(p) || row0 < 0 || row1 > p->N || row0 >= row1) return ORC_BAD;
-  orc_attn_in in = {NULL, NULL, NULL, NULL, NULL, NULL, NULL, q, k, v};
+  orc_attn_in in = {NULL, NULL, NULL, NULL, NULL, NULL, NULL, q, k, v, NULL, row0};
   attn_rows(p, &in, 0, row0, row1, out, lse, NULL, NULL, NULL);
   return ORC_OK;
 }

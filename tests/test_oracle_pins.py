@@ -372,3 +372,34 @@ def test_half_rotation_beats_no_rotation(orc):
         ref = orc.reference_attention_fp64(h["q_rot"], h["k_rot"], x["v"][0, 0])
         cos[rot] = _cosine(r["out"], ref)
     assert cos[2] > cos[0]
+
+
+def test_given_codes_entry(orc):
+    """Attention on supplied P codes: its own codes reproduce it exactly; a
+    flipped code changes the output as the unblocked closed form says."""
+    wl, p, x, h = _head(orc, "small")
+    R = 64
+    r = orc.attention_int4_rows(p, h, 0, R, dumps=True)
+    same = orc.attention_int4_rows_given_codes(p, h, r["codes"], 0, R)
+    assert np.array_equal(same["out"], r["out"]) and np.array_equal(same["lse"], r["lse"])
+    codes = r["codes"].copy()
+    i, j = 5, int(np.nonzero(codes[5] < 7)[0][0])
+    codes[i, j] += 1
+    flipped = orc.attention_int4_rows_given_codes(p, h, codes, 0, R)["out"]
+    # closed form with the flipped code
+    ref, ref_codes = _brute_force_quantised(wl, h, np.arange(R))
+    from oracle import unpack_codes
+    v = unpack_codes(h["v4"]).astype(np.float64) * h["sv"].astype(np.float64)
+    q = unpack_codes(h["q4"]).astype(np.int64)
+    k = unpack_codes(h["k4"]).astype(np.int64)
+    ci = np.float32(h["sq"][i]) * np.float32(1.0 / math.sqrt(wl.D))
+    S = ((q[i] @ k.T).astype(np.float32) * h["sk"].astype(np.float32)) * ci
+    Bk = wl.block_k
+    nb = -(-wl.N // Bk)
+    run = np.maximum.accumulate(np.array([S[t * Bk:(t + 1) * Bk].max() for t in range(nb)]))
+    M = np.repeat(run, Bk)[:wl.N].astype(np.float64)
+    w = np.exp(M - run[-1]) * (codes[i].astype(np.float64) + 8)
+    expect = (w @ v) / w.sum()
+    assert np.abs(flipped[i] - expect).max() <= 1e-12 * np.abs(expect).max()
+    others = np.arange(R) != i
+    assert np.array_equal(flipped[others], r["out"][others])
