@@ -40,6 +40,8 @@ namespace ra {
 namespace {
 
 __device__ uint32_t g_attn_status = 0;
+// First timed-out wait: (site << 24) | (block counter & 0xFFFF) << 8 | (cta & 0xFF).
+__device__ uint32_t g_attn_diag = 0;
 
 constexpr int kThreads = 384;
 constexpr int kRows = 128;          // query rows per tile = MMA M
@@ -65,7 +67,7 @@ struct Cfg {
   static constexpr int oPk = oVw + kVS * ((kVwBytes + 1023) / 1024) * 1024;
   static constexpr int oKsc = oPk + kPS * 2 * kPkHalf;
   static constexpr int oBar = oKsc + kKS * BN * 4;
-  static constexpr int kNumBars = 4 + 2 * kPS + 2 * kKS + 2 * kVS + 4 + 4 + 2 + 1;
+  static constexpr int kNumBars = 4 + 2 * kPS + 2 * kKS + 2 * kVS + 4 + 4 + 4 + 1;
   static constexpr int oMisc = oBar + kNumBars * 8;
   static constexpr int kSmem = oMisc + 16 + 1024;       // + alignment slack
   static constexpr int kKwStride = ((kKwBytes + 1023) / 1024) * 1024;
@@ -84,7 +86,7 @@ struct Bars {
   uint64_t* vw_full; uint64_t* vw_empty;
   uint64_t* s_full;   // [tile][buf]
   uint64_t* p_full;   // [tile][buf]
-  uint64_t* pv_done;  // [tile]
+  uint64_t* pv_done;  // [tile][buf]: P.V of the blocks whose P sits in S buffer buf
   uint64_t* drain;
 };
 
@@ -136,6 +138,18 @@ __device__ __forceinline__ float max3(float a, float b, float c) { return fmaxf(
 
 __device__ __forceinline__ void set_status(uint32_t bits) { atomicOr(&g_attn_status, bits); }
 
+// Records the first wait that gave up (site id, block counter, CTA) for diagnosis.
+__device__ __forceinline__ void note_timeout(uint32_t site, uint32_t g) {
+  atomicCAS(&g_attn_diag, 0u, (site << 24) | ((g & 0xFFFFu) << 8) | (blockIdx.x & 0xFFu));
+}
+
+__device__ __forceinline__ bool wait_at(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t site,
+                                        uint32_t g) {
+  const int r = mbar_wait_ex(bar, parity, abort);
+  if (r < 0) note_timeout(site, g);
+  return r > 0;
+}
+
 template <int D, int BN, bool DUMP>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -151,7 +165,7 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     B.pk_full = b; b += C::kPS; B.pk_empty = b; b += C::kPS;
     B.kw_full = b; b += C::kKS; B.kw_empty = b; b += C::kKS;
     B.vw_full = b; b += C::kVS; B.vw_empty = b; b += C::kVS;
-    B.s_full = b; b += 4; B.p_full = b; b += 4; B.pv_done = b; b += 2; B.drain = b; b += 1;
+    B.s_full = b; b += 4; B.p_full = b; b += 4; B.pv_done = b; b += 4; B.drain = b; b += 1;
   }
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::oMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::oMisc + 4);
@@ -162,8 +176,8 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     for (int s = 0; s < C::kPS; ++s) { mbar_init(B.pk_full + s, 1); mbar_init(B.pk_empty + s, 2); }
     for (int s = 0; s < C::kKS; ++s) { mbar_init(B.kw_full + s, 2); mbar_init(B.kw_empty + s, 1 + 8); }
     for (int s = 0; s < C::kVS; ++s) { mbar_init(B.vw_full + s, 2); mbar_init(B.vw_empty + s, 1); }
-    for (int s = 0; s < 4; ++s) { mbar_init(B.s_full + s, 1); mbar_init(B.p_full + s, 4); }
-    mbar_init(B.pv_done + 0, 1); mbar_init(B.pv_done + 1, 1); mbar_init(B.drain, 1);
+    for (int s = 0; s < 4; ++s) { mbar_init(B.s_full + s, 1); mbar_init(B.p_full + s, 4); mbar_init(B.pv_done + s, 1); }
+    mbar_init(B.drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -189,14 +203,14 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         bool ok = true;
         for (int item = blockIdx.x; item < prm.nitems && ok; item += gridDim.x, ++li) {
           const int bh = item / prm.npairs, pair = item % prm.npairs;
-          ok = mbar_wait(B.qpk_empty, (li & 1) ^ 1, abort_flag);
+          ok = wait_at(B.qpk_empty, (li & 1) ^ 1, abort_flag, 1u, li);
           if (!ok) break;
           mbar_arrive_expect_tx(B.qpk_full, kTiles * C::kQPkBytes);
           for (int tt = 0; tt < kTiles; ++tt)
             tma_load_3d(smem + C::oQPk + tt * C::kQPkBytes, &tm_q, B.qpk_full, 0, pair * 2 * kRows + tt * kRows, bh);
           for (int t = 0; t < nb; ++t, ++g) {
             const int s = g % C::kPS;
-            ok = mbar_wait(B.pk_empty + s, ((g / C::kPS) & 1) ^ 1, abort_flag);
+            ok = wait_at(B.pk_empty + s, ((g / C::kPS) & 1) ^ 1, abort_flag, 14u, g);
             if (!ok) break;
             mbar_arrive_expect_tx(B.pk_full + s, 2 * C::kPkHalf);
             uint8_t* dst = smem + C::oPk + s * 2 * C::kPkHalf;
@@ -222,10 +236,10 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         bool ok = true;
         auto issue_pv = [&](uint32_t gg) -> bool {
           const int vs = gg % C::kVS;
-          if (!mbar_wait(B.vw_full + vs, (gg / C::kVS) & 1, abort_flag)) return false;
+          if (!wait_at(B.vw_full + vs, (gg / C::kVS) & 1, abort_flag, 2u, gg)) return false;
           const uint32_t buf = gg & 1;
           for (int tt = 0; tt < kTiles; ++tt) {
-            if (!mbar_wait(B.p_full + tt * 2 + buf, (gg >> 1) & 1, abort_flag)) return false;
+            if (!wait_at(B.p_full + tt * 2 + buf, (gg >> 1) & 1, abort_flag, 3u, gg)) return false;
             tc_fence_after();
             const uint32_t tP = tbase + tt * 256 + buf * 64;
             const uint32_t tA = tbase + tt * 256 + 128;
@@ -235,22 +249,32 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                                                8 * D, C::kSwz);
               mma_i8_ts(tA, tP + kk * 8, bdesc, C::kIdescPV, 1);
             }
-            mma_commit(B.pv_done + tt);
+            mma_commit(B.pv_done + tt * 2 + buf);
           }
           mma_commit(B.vw_empty + vs);
           return true;
         };
         for (int item = blockIdx.x; item < prm.nitems && ok; item += gridDim.x, ++li) {
-          ok = mbar_wait(B.q_full, li & 1, abort_flag);
+          ok = wait_at(B.q_full, li & 1, abort_flag, 4u, li);
           if (!ok) break;
           tc_fence_after();
           for (int t = 0; t < nb && ok; ++t, ++g) {
             const int ks = g % C::kKS;
-            ok = mbar_wait(B.kw_full + ks, (g / C::kKS) & 1, abort_flag);
+            ok = wait_at(B.kw_full + ks, (g / C::kKS) & 1, abort_flag, 5u, g);
             if (!ok) break;
             tc_fence_after();
             const uint32_t buf = g & 1;
             for (int tt = 0; tt < kTiles; ++tt) {
+              // P(g-2) of this tile lives in the S buffer QK(g) overwrites, and
+              // MMAs into different accumulators are not ordered by the tensor
+              // pipe: wait until P.V of block g-2 has read it.  pv_done has one
+              // barrier per S buffer, so P.V(g-4), the previous completion on
+              // it, is done (QK(g-2) waited for it) and the awaited phase is
+              // the barrier's current one.
+              if (g >= 2) {
+                if (!(ok = wait_at(B.pv_done + tt * 2 + buf, ((g - 2) >> 1) & 1, abort_flag, 6u, g))) break;
+                tc_fence_after();
+              }
               const uint32_t tS = tbase + tt * 256 + buf * 64;
 #pragma unroll
               for (int kk = 0; kk < D / 32; ++kk) {
@@ -260,6 +284,7 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
               }
               mma_commit(B.s_full + tt * 2 + buf);
             }
+            if (!ok) break;
             mma_commit(B.kw_empty + ks);
             if (t == nb - 1) mma_commit(B.q_free);
             if (t > 0) ok = issue_pv(g - 1);
@@ -279,8 +304,8 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       bool ok = true;
       for (int item = blockIdx.x; item < prm.nitems && ok; item += gridDim.x, ++li) {
         const int bh = item / prm.npairs;
-        if (!(ok = mbar_wait(B.qpk_full, li & 1, abort_flag))) break;
-        if (!(ok = mbar_wait(B.q_free, (li & 1) ^ 1, abort_flag))) break;
+        if (!(ok = wait_at(B.qpk_full, li & 1, abort_flag, 7u, li))) break;
+        if (!(ok = wait_at(B.q_free, (li & 1) ^ 1, abort_flag, 8u, li))) break;
         for (int tt = 0; tt < kTiles; ++tt)
           widen_tile<D>(smem + C::oQPk + tt * C::kQPkBytes, smem + C::oQ + tt * C::kQBytes, kRows, wt, 64);
         fence_proxy_async_smem();
@@ -288,8 +313,8 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (lane == 0) { mbar_arrive(B.qpk_empty); mbar_arrive(B.q_full); }
         for (int t = 0; t < nb; ++t, ++g) {
           const int s = g % C::kPS, ks = g % C::kKS, vs = g % C::kVS;
-          if (!(ok = mbar_wait(B.pk_full + s, (g / C::kPS) & 1, abort_flag))) break;
-          if (!(ok = mbar_wait(B.kw_empty + ks, ((g / C::kKS) & 1) ^ 1, abort_flag))) break;
+          if (!(ok = wait_at(B.pk_full + s, (g / C::kPS) & 1, abort_flag, 9u, g))) break;
+          if (!(ok = wait_at(B.kw_empty + ks, ((g / C::kKS) & 1) ^ 1, abort_flag, 15u, g))) break;
           const uint8_t* pk = smem + C::oPk + s * 2 * C::kPkHalf;
           widen_tile<D>(pk, smem + C::oKw + ks * C::kKwStride, BN, wt, 64);
           if (wt < BN) {
@@ -300,7 +325,7 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) mbar_arrive(B.kw_full + ks);
-          if (!(ok = mbar_wait(B.vw_empty + vs, ((g / C::kVS) & 1) ^ 1, abort_flag))) break;
+          if (!(ok = wait_at(B.vw_empty + vs, ((g / C::kVS) & 1) ^ 1, abort_flag, 16u, g))) break;
           widen_tile<D>(pk + C::kPkHalf, smem + C::oVw + vs * C::kVwStride, BN, wt, 64);
           fence_proxy_async_smem();
           __syncwarp();
@@ -339,14 +364,14 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       for (int t = 0; t < nb; ++t, ++g) {
         const uint32_t buf = g & 1;
         const uint32_t tS = tbase + tt * 256 + buf * 64 + lane_off;
-        if (!(ok = mbar_wait(B.s_full + tt * 2 + buf, (g >> 1) & 1, abort_flag))) break;
+        if (!(ok = wait_at(B.s_full + tt * 2 + buf, (g >> 1) & 1, abort_flag, 10u, g))) break;
+        __syncwarp();
         tc_fence_after();
         uint32_t raw[BN];
         tmem_ld<BN>(tS, raw);
         const int ks = g % C::kKS;
-        if (!(ok = mbar_wait(B.kw_full + ks, (g / C::kKS) & 1, abort_flag))) break;
+        if (!(ok = wait_at(B.kw_full + ks, (g / C::kKS) & 1, abort_flag, 11u, g))) break;
         const float* ksc = reinterpret_cast<const float*>(smem + C::oKsc) + ks * BN;
-        tmem_wait_ld();
         const int nvalid = min(BN, prm.N - t * BN);
         float v[BN];
 #pragma unroll
@@ -401,13 +426,13 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const bool near_bound = (Lrun + 15 * BN) * 112 >= (1 << 22) - 4096;
         const bool need = (t > 0) && (grow || near_bound || DUMP);
         if (__any_sync(0xFFFFFFFFu, need)) {
-          if (!(ok = mbar_wait(B.pv_done + tt, (g - 1) & 1, abort_flag))) break;
+          if (!(ok = wait_at(B.pv_done + tt * 2 + ((g - 1) & 1), ((g - 1) >> 1) & 1, abort_flag, 12u, g))) break;
+          __syncwarp();
           tc_fence_after();
 #pragma unroll
           for (int c = 0; c < D; c += 32) {
             uint32_t a[32];
             tmem_ld32(tA + c, a);
-            tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
               const float af = __int_as_float(static_cast<int>(a[i])) - kMagicF;
@@ -439,7 +464,6 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         Lrun += lq;
         m_run = m_new;
-        tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
@@ -449,13 +473,13 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       }
       if (!ok) break;
       // Last block: fold the accumulator, normalise, store.
-      if (!(ok = mbar_wait(B.pv_done + tt, (g - 1) & 1, abort_flag))) break;
+      if (!(ok = wait_at(B.pv_done + tt * 2 + ((g - 1) & 1), ((g - 1) >> 1) & 1, abort_flag, 13u, g))) break;
+      __syncwarp();
       tc_fence_after();
 #pragma unroll
       for (int c = 0; c < D; c += 32) {
         uint32_t a[32];
         tmem_ld32(tA + c, a);
-        tmem_wait_ld();
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           const float af = __int_as_float(static_cast<int>(a[i])) - kMagicF;
@@ -579,6 +603,13 @@ cudaError_t launch_attn_int4(const ra_problem& p, const uint8_t* q4, const float
 #undef RA_CASE
   *unsupported = 1;
   return cudaSuccess;
+}
+
+cudaError_t read_attn_int4_diag(uint32_t* out) {
+  uint32_t zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(out, g_attn_diag, sizeof(uint32_t));
+  if (e != cudaSuccess) return e;
+  return cudaMemcpyToSymbol(g_attn_diag, &zero, sizeof(uint32_t));
 }
 
 cudaError_t read_attn_int4_status(uint32_t* out) {
