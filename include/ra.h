@@ -179,6 +179,35 @@ ra_status ra_attn_bf16_fallback(const ra_problem* p, const void* q, const void* 
                                 const void* v, void* out, float* lse, void* stream);
 
 /*
+ * Allocation-free prologue.  (The paper has no counterpart; this is a
+ * deployment convenience.)  Same computation, arguments and results as
+ * ra_rope_rotate_quant, without the workspace arguments: it is meant for
+ * callers that cannot allocate device memory when they run it, such as an
+ * inference-engine plugin whose execute step may not call the allocator, or a
+ * service with a fixed device-memory budget reserved at start-up.
+ *
+ * The scratch space is a fixed array of RA_STATIC_SCRATCH_BYTES inside the
+ * library's device memory; every GPU that loads the library holds it until the
+ * process exits.  The entry point never allocates or frees memory.
+ *   - Problems whose ra_workspace_bytes(p) exceeds RA_STATIC_SCRATCH_BYTES
+ *     return RA_ERR_UNSUPPORTED and launch nothing (32 MiB covers, e.g.,
+ *     B*H*ceil(N/256) <= ~21000 at D = 128).
+ *   - The first call on a device looks up the array's device address, with
+ *     that device current; make that first call before any stream capture.
+ *   - All calls on a device share the one array: calls whose work may overlap
+ *     on the GPU (different streams without ordering between them) race on it.
+ *     Calls ordered on one stream are safe; the array keeps the last call's
+ *     contents, and nothing in it needs to start at zero.
+ */
+#define RA_STATIC_SCRATCH_BYTES ((size_t)32 << 20)
+ra_status ra_rope_rotate_quant_noalloc(const ra_problem* p, int in_dtype,
+                                       const void* q, const void* k, const void* v,
+                                       const int32_t* pos,
+                                       uint8_t* q4, float* sq, uint8_t* k4, float* sk,
+                                       float* k_mean, uint8_t* v4, float* sv, int32_t* v_colsum,
+                                       void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device status word of the
  * current device.  Returns RA_OK, RA_ERR_INVALID_ARG (a kernel saw a position
  * outside the grid), RA_ERR_TIMEOUT (an internal wait ran past its bound) or

@@ -222,3 +222,30 @@ def attn_bf16_fallback(p: Problem, q: torch.Tensor, k: torch.Tensor, v: torch.Te
 def sync_status(stream=None) -> int:
     """ra_sync_status: synchronises the stream and returns (and clears) the device status."""
     return int(lib().ra_sync_status(C.c_void_p(_stream(stream))))
+
+
+def rope_rotate_quant_noalloc(p: Problem, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, pos: torch.Tensor,
+                              out: Dict[str, torch.Tensor], stream=None) -> Dict[str, torch.Tensor]:
+    """ra_rope_rotate_quant_noalloc: the prologue without a workspace argument.
+
+    For callers that cannot allocate device memory while they run (the library
+    keeps a fixed scratch array of RA_STATIC_SCRATCH_BYTES per GPU instead).  The
+    caller supplies every output tensor in `out` (keys as rope_rotate_quant
+    returns).  The first call on a device should precede any stream capture, and
+    calls that may overlap on the GPU share, and race on, the one scratch array.
+    """
+    L = lib()
+    fn = L.ra_rope_rotate_quant_noalloc
+    fn.restype = C.c_int
+    fn.argtypes = [C.POINTER(Problem), C.c_int] + [C.c_void_p] * 13
+    B, H, N, D = p.B, p.H, p.N, p.D
+    shp = (B, H, N, D)
+    rc = fn(C.byref(p), _in_dtype(q), _ptr(q, q.dtype, shp, "q"), _ptr(k, q.dtype, shp, "k"),
+            _ptr(v, q.dtype, shp, "v"), _ptr(pos, torch.int32, (N, 3), "pos"),
+            _ptr(out["q4"], torch.uint8, (B, H, N, D // 2)), _ptr(out["sq"], torch.float32, (B, H, N)),
+            _ptr(out["k4"], torch.uint8, (B, H, N, D // 2)), _ptr(out["sk"], torch.float32, (B, H, N)),
+            _ptr(out["k_mean"], torch.float32, (B, H, D)), _ptr(out["v4"], torch.uint8, (B, H, N, D // 2)),
+            _ptr(out["sv"], torch.float32, (B, H, D)), _ptr(out["v_colsum"], torch.int32, (B, H, _nblocks(p), D)),
+            C.c_void_p(_stream(stream)))
+    _check("ra_rope_rotate_quant_noalloc", rc)
+    return out
