@@ -43,7 +43,7 @@ __device__ uint32_t g_attn_status = 0;
 // First timed-out wait: (site << 24) | (block counter & 0xFFFF) << 8 | (cta & 0xFF).
 __device__ uint32_t g_attn_diag = 0;
 
-constexpr int kThreads = 384;
+constexpr int kThreads = 512;   // 16 warps: see the role map in the kernel
 constexpr int kRows = 128;          // query rows per tile = MMA M
 constexpr int kTiles = 2;           // query tiles per CTA
 constexpr uint32_t kMagic = 0x4B400000u;  // bits of 1.5 * 2^23
@@ -66,8 +66,12 @@ struct Cfg {
   static constexpr int oVw = oKw + kKS * ((kKwBytes + 1023) / 1024) * 1024;
   static constexpr int oPk = oVw + kVS * ((kVwBytes + 1023) / 1024) * 1024;
   static constexpr int oKsc = oPk + kPS * 2 * kPkHalf;
-  static constexpr int oBar = oKsc + kKS * BN * 4;
-  static constexpr int kNumBars = 4 + 2 * kPS + 2 * kKS + 2 * kVS + 4 + 4 + 4 + 1;
+  // Half of every softmax row's fp32 output accumulator lives in shared
+  // memory (the other half in registers); rows padded to avoid bank conflicts.
+  static constexpr int kFRow = D / 2 + 4;                 // floats per row
+  static constexpr int oF = oKsc + kKS * BN * 4;
+  static constexpr int oBar = oF + kTiles * kRows * kFRow * 4;
+  static constexpr int kNumBars = 4 + 2 * kPS + 2 * kKS + 2 * kVS + 4 + 4 + 4 + 2;
   static constexpr int oMisc = oBar + kNumBars * 8;
   static constexpr int kSmem = oMisc + 16 + 1024;       // + alignment slack
   static constexpr int kKwStride = ((kKwBytes + 1023) / 1024) * 1024;
@@ -87,7 +91,7 @@ struct Bars {
   uint64_t* s_full;   // [tile][buf]
   uint64_t* p_full;   // [tile][buf]
   uint64_t* pv_done;  // [tile][buf]: P.V of the blocks whose P sits in S buffer buf
-  uint64_t* drain;
+  uint64_t* drain;    // [issuer]
 };
 
 struct AttnParams {
@@ -144,8 +148,8 @@ __device__ __forceinline__ void note_timeout(uint32_t site, uint32_t g) {
 }
 
 __device__ __forceinline__ bool wait_at(uint64_t* bar, uint32_t parity, volatile int* abort, uint32_t site,
-                                        uint32_t g) {
-  const int r = mbar_wait_ex(bar, parity, abort);
+                                        uint32_t g, uint32_t backoff_ns = 16) {
+  const int r = mbar_wait_ex(bar, parity, abort, backoff_ns);
   if (r < 0) note_timeout(site, g);
   return r > 0;
 }
@@ -156,7 +160,9 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                  const __grid_constant__ CUtensorMap tm_v, const AttnParams prm) {
   using C = Cfg<D, BN>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte aligned base; pointer arithmetic on the shared array keeps the
+  // shared address space visible to the compiler (LDS/STS, not generic LD/ST).
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::oBar);
   Bars B;
   {
@@ -165,19 +171,20 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     B.pk_full = b; b += C::kPS; B.pk_empty = b; b += C::kPS;
     B.kw_full = b; b += C::kKS; B.kw_empty = b; b += C::kKS;
     B.vw_full = b; b += C::kVS; B.vw_empty = b; b += C::kVS;
-    B.s_full = b; b += 4; B.p_full = b; b += 4; B.pv_done = b; b += 4; B.drain = b; b += 1;
+    B.s_full = b; b += 4; B.p_full = b; b += 4; B.pv_done = b; b += 4; B.drain = b; b += 2;
   }
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::oMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::oMisc + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    mbar_init(B.qpk_full, 1); mbar_init(B.qpk_empty, 2); mbar_init(B.q_full, 2); mbar_init(B.q_free, 1);
-    for (int s = 0; s < C::kPS; ++s) { mbar_init(B.pk_full + s, 1); mbar_init(B.pk_empty + s, 2); }
-    for (int s = 0; s < C::kKS; ++s) { mbar_init(B.kw_full + s, 2); mbar_init(B.kw_empty + s, 1 + 8); }
-    for (int s = 0; s < C::kVS; ++s) { mbar_init(B.vw_full + s, 2); mbar_init(B.vw_empty + s, 1); }
+    mbar_init(B.qpk_full, 1); mbar_init(B.qpk_empty, 4); mbar_init(B.q_full, 4); mbar_init(B.q_free, 2);
+    for (int s = 0; s < C::kPS; ++s) { mbar_init(B.pk_full + s, 1); mbar_init(B.pk_empty + s, 4); }
+    for (int s = 0; s < C::kKS; ++s) { mbar_init(B.kw_full + s, 4); mbar_init(B.kw_empty + s, 2 + 8); }
+    for (int s = 0; s < C::kVS; ++s) { mbar_init(B.vw_full + s, 4); mbar_init(B.vw_empty + s, 2); }
     for (int s = 0; s < 4; ++s) { mbar_init(B.s_full + s, 1); mbar_init(B.p_full + s, 4); mbar_init(B.pv_done + s, 1); }
     mbar_init(B.drain, 1);
+    mbar_init(B.drain + 1, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -194,8 +201,12 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const uint32_t tbase = *tmem_holder;
 
   const int nb = prm.nblocks;
-  if (warp < 4) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
+  // Roles: warp 0 TMA producer, warp 1 MMA issuer of tile 0 and TMEM owner,
+  // warp 2 MMA issuer of tile 1, warp 3 idle, warps 4-7 widen codes (one per
+  // SM sub-partition), warps 8-11 and 12-15 softmax of query tiles 0 and 1.
+  if (warp < 8) {
+    if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 56;");
+    else asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
     if (warp == 0) {
       // ------------------------------------------------------------ TMA producer
       if (lane == 0) {
@@ -203,14 +214,14 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         bool ok = true;
         for (int item = blockIdx.x; item < prm.nitems && ok; item += gridDim.x, ++li) {
           const int bh = item / prm.npairs, pair = item % prm.npairs;
-          ok = wait_at(B.qpk_empty, (li & 1) ^ 1, abort_flag, 1u, li);
+          ok = wait_at(B.qpk_empty, (li & 1) ^ 1, abort_flag, 1u, li, 256u);
           if (!ok) break;
           mbar_arrive_expect_tx(B.qpk_full, kTiles * C::kQPkBytes);
           for (int tt = 0; tt < kTiles; ++tt)
             tma_load_3d(smem + C::oQPk + tt * C::kQPkBytes, &tm_q, B.qpk_full, 0, pair * 2 * kRows + tt * kRows, bh);
           for (int t = 0; t < nb; ++t, ++g) {
             const int s = g % C::kPS;
-            ok = wait_at(B.pk_empty + s, ((g / C::kPS) & 1) ^ 1, abort_flag, 14u, g);
+            ok = wait_at(B.pk_empty + s, ((g / C::kPS) & 1) ^ 1, abort_flag, 14u, g, 256u);
             if (!ok) break;
             mbar_arrive_expect_tx(B.pk_full + s, 2 * C::kPkHalf);
             uint8_t* dst = smem + C::oPk + s * 2 * C::kPkHalf;
@@ -226,23 +237,56 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         if (!ok) set_status(kStatusTimeout);
       }
-    } else if (warp == 1) {
-      // ------------------------------------------------------------ MMA issuer
+    } else if (warp == 1 || warp == 2) {
+      // ------------------------------------------------------------ MMA issuers
+      // One issuing thread per query tile, so each tile's pipeline advances at
+      // its own pace (within the shared K/V stage window).  Per tile: P.V(g),
+      // then QK(g+2) into the S buffer whose P codes P.V(g) has just read.
       if (lane == 0) {
-        const uint32_t sQ = smem_u32(smem + C::oQ);
+        const int tt = warp - 1;
+        const uint32_t sQ = smem_u32(smem + C::oQ) + tt * C::kQBytes;
         const uint32_t sKw = smem_u32(smem + C::oKw);
         const uint32_t sVw = smem_u32(smem + C::oVw);
-        uint32_t g = 0, li = 0;
+        const uint32_t tS0 = tbase + tt * 256;
+        const uint32_t tA = tS0 + 128;
+        uint32_t li = 0, g0 = 0;
         bool ok = true;
-        auto issue_pv = [&](uint32_t gg) -> bool {
-          const int vs = gg % C::kVS;
-          if (!wait_at(B.vw_full + vs, (gg / C::kVS) & 1, abort_flag, 2u, gg)) return false;
-          const uint32_t buf = gg & 1;
-          for (int tt = 0; tt < kTiles; ++tt) {
-            if (!wait_at(B.p_full + tt * 2 + buf, (gg >> 1) & 1, abort_flag, 3u, gg)) return false;
+        // QK(gq) into S buffer gq & 1; before that, P.V(gq - 2) (which reads the
+        // P codes stored in that buffer) must have completed.  pv_done has one
+        // barrier per S buffer, so P.V(gq - 4), the previous completion on it,
+        // is done and the awaited phase is the barrier's current one.
+        auto issue_qk = [&](uint32_t gq, bool last_of_item) -> bool {
+          const uint32_t buf = gq & 1;
+          if (gq >= 2) {
+            if (!wait_at(B.pv_done + tt * 2 + buf, ((gq - 2) >> 1) & 1, abort_flag, 6u, gq, 32u)) return false;
+          }
+          const int ks = gq % C::kKS;
+          if (!wait_at(B.kw_full + ks, (gq / C::kKS) & 1, abort_flag, 5u, gq, 32u)) return false;
+          tc_fence_after();
+          const uint32_t tS = tS0 + buf * 64;
+#pragma unroll
+          for (int kk = 0; kk < D / 32; ++kk) {
+            const uint64_t adesc = smem_desc(sQ + kk * 32, 16, 8 * D, C::kSwz);
+            const uint64_t bdesc = smem_desc(sKw + ks * C::kKwStride + kk * 32, 16, 8 * D, C::kSwz);
+            mma_i8_ss(tS, adesc, bdesc, C::kIdescQK, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(B.s_full + tt * 2 + buf);
+          mma_commit(B.kw_empty + ks);
+          if (last_of_item) mma_commit(B.q_free);
+          return true;
+        };
+        for (int item = blockIdx.x; item < prm.nitems && ok; item += gridDim.x, ++li, g0 += nb) {
+          if (!(ok = wait_at(B.q_full, li & 1, abort_flag, 4u, li, 32u))) break;
+          tc_fence_after();
+          for (int t = 0; t < 2 && t < nb && ok; ++t) ok = issue_qk(g0 + t, t == nb - 1);
+          for (int t = 0; t < nb && ok; ++t) {
+            const uint32_t gg = g0 + t;
+            const int vs = gg % C::kVS;
+            const uint32_t buf = gg & 1;
+            if (!(ok = wait_at(B.vw_full + vs, (gg / C::kVS) & 1, abort_flag, 2u, gg, 32u))) break;
+            if (!(ok = wait_at(B.p_full + tt * 2 + buf, (gg >> 1) & 1, abort_flag, 3u, gg, 32u))) break;
             tc_fence_after();
-            const uint32_t tP = tbase + tt * 256 + buf * 64;
-            const uint32_t tA = tbase + tt * 256 + 128;
+            const uint32_t tP = tS0 + buf * 64;
 #pragma unroll
             for (int kk = 0; kk < C::kKeysPV / 32; ++kk) {
               const uint64_t bdesc = smem_desc(sVw + vs * C::kVwStride + kk * 32 * D, 8 * D * (C::kKeysPV / 8),
@@ -250,83 +294,49 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
               mma_i8_ts(tA, tP + kk * 8, bdesc, C::kIdescPV, 1);
             }
             mma_commit(B.pv_done + tt * 2 + buf);
+            mma_commit(B.vw_empty + vs);
+            if (t + 2 < nb) ok = issue_qk(gg + 2, t + 2 == nb - 1);
           }
-          mma_commit(B.vw_empty + vs);
-          return true;
-        };
-        for (int item = blockIdx.x; item < prm.nitems && ok; item += gridDim.x, ++li) {
-          ok = wait_at(B.q_full, li & 1, abort_flag, 4u, li);
-          if (!ok) break;
-          tc_fence_after();
-          for (int t = 0; t < nb && ok; ++t, ++g) {
-            const int ks = g % C::kKS;
-            ok = wait_at(B.kw_full + ks, (g / C::kKS) & 1, abort_flag, 5u, g);
-            if (!ok) break;
-            tc_fence_after();
-            const uint32_t buf = g & 1;
-            for (int tt = 0; tt < kTiles; ++tt) {
-              // P(g-2) of this tile lives in the S buffer QK(g) overwrites, and
-              // MMAs into different accumulators are not ordered by the tensor
-              // pipe: wait until P.V of block g-2 has read it.  pv_done has one
-              // barrier per S buffer, so P.V(g-4), the previous completion on
-              // it, is done (QK(g-2) waited for it) and the awaited phase is
-              // the barrier's current one.
-              if (g >= 2) {
-                if (!(ok = wait_at(B.pv_done + tt * 2 + buf, ((g - 2) >> 1) & 1, abort_flag, 6u, g))) break;
-                tc_fence_after();
-              }
-              const uint32_t tS = tbase + tt * 256 + buf * 64;
-#pragma unroll
-              for (int kk = 0; kk < D / 32; ++kk) {
-                const uint64_t adesc = smem_desc(sQ + tt * C::kQBytes + kk * 32, 16, 8 * D, C::kSwz);
-                const uint64_t bdesc = smem_desc(sKw + ks * C::kKwStride + kk * 32, 16, 8 * D, C::kSwz);
-                mma_i8_ss(tS, adesc, bdesc, C::kIdescQK, kk > 0 ? 1u : 0u);
-              }
-              mma_commit(B.s_full + tt * 2 + buf);
-            }
-            if (!ok) break;
-            mma_commit(B.kw_empty + ks);
-            if (t == nb - 1) mma_commit(B.q_free);
-            if (t > 0) ok = issue_pv(g - 1);
-          }
-          if (ok) ok = issue_pv(g - 1);
         }
-        // Drain: every MMA issued so far has completed before TMEM is released.
-        mma_commit(B.drain);
+        // Drain: every MMA issued by this thread has completed before TMEM is released.
+        mma_commit(B.drain + tt);
         uint32_t it = 0;
-        while (!mbar_try_wait(B.drain, 0) && ++it < kSpinLimit) {}
+        while (!mbar_try_wait(B.drain + tt, 0) && ++it < kSpinLimit) {}
         if (!ok) set_status(kStatusTimeout);
       }
-    } else {
+    } else if (warp >= 4) {
       // ------------------------------------------------------------ widening warps
-      const int wt = threadIdx.x - 64;  // 0..63
+      const int wt = threadIdx.x - 128;  // 0..127
       uint32_t g = 0, li = 0;
       bool ok = true;
       for (int item = blockIdx.x; item < prm.nitems && ok; item += gridDim.x, ++li) {
         const int bh = item / prm.npairs;
-        if (!(ok = wait_at(B.qpk_full, li & 1, abort_flag, 7u, li))) break;
-        if (!(ok = wait_at(B.q_free, (li & 1) ^ 1, abort_flag, 8u, li))) break;
+        if (!(ok = wait_at(B.qpk_full, li & 1, abort_flag, 7u, li, 256u))) break;
+        if (!(ok = wait_at(B.q_free, (li & 1) ^ 1, abort_flag, 8u, li, 256u))) break;
         for (int tt = 0; tt < kTiles; ++tt)
-          widen_tile<D>(smem + C::oQPk + tt * C::kQPkBytes, smem + C::oQ + tt * C::kQBytes, kRows, wt, 64);
+          widen_tile<D>(smem + C::oQPk + tt * C::kQPkBytes, smem + C::oQ + tt * C::kQBytes, kRows, wt, 128);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) { mbar_arrive(B.qpk_empty); mbar_arrive(B.q_full); }
         for (int t = 0; t < nb; ++t, ++g) {
           const int s = g % C::kPS, ks = g % C::kKS, vs = g % C::kVS;
-          if (!(ok = wait_at(B.pk_full + s, (g / C::kPS) & 1, abort_flag, 9u, g))) break;
-          if (!(ok = wait_at(B.kw_empty + ks, ((g / C::kKS) & 1) ^ 1, abort_flag, 15u, g))) break;
+          if (!(ok = wait_at(B.pk_full + s, (g / C::kPS) & 1, abort_flag, 9u, g, 128u))) break;
+          if (!(ok = wait_at(B.kw_empty + ks, ((g / C::kKS) & 1) ^ 1, abort_flag, 15u, g, 256u))) break;
           const uint8_t* pk = smem + C::oPk + s * 2 * C::kPkHalf;
-          widen_tile<D>(pk, smem + C::oKw + ks * C::kKwStride, BN, wt, 64);
+          widen_tile<D>(pk, smem + C::oKw + ks * C::kKwStride, BN, wt, 128);
           if (wt < BN) {
             const int j = t * BN + wt;
             float* ksc = reinterpret_cast<float*>(smem + C::oKsc) + ks * BN;
-            ksc[wt] = j < prm.N ? prm.sk[static_cast<size_t>(bh) * prm.N + j] * (1.0f / 256.0f) : 0.0f;
+            // Keys past N get a NaN scale: their score is NaN, which the
+            // maximum ignores, and their code bytes are masked in the softmax.
+            ksc[wt] = j < prm.N ? prm.sk[static_cast<size_t>(bh) * prm.N + j] * (1.0f / 256.0f)
+                                : __int_as_float(0x7FC00000);
           }
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) mbar_arrive(B.kw_full + ks);
-          if (!(ok = wait_at(B.vw_empty + vs, ((g / C::kVS) & 1) ^ 1, abort_flag, 16u, g))) break;
-          widen_tile<D>(pk + C::kPkHalf, smem + C::oVw + vs * C::kVwStride, BN, wt, 64);
+          if (!(ok = wait_at(B.vw_empty + vs, ((g / C::kVS) & 1) ^ 1, abort_flag, 16u, g, 256u))) break;
+          widen_tile<D>(pk + C::kPkHalf, smem + C::oVw + vs * C::kVwStride, BN, wt, 128);
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) { mbar_arrive(B.vw_full + vs); mbar_arrive(B.pk_empty + s); }
@@ -335,17 +345,50 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       if (!ok) set_status(kStatusTimeout);
     }
   } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 232;");
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 208;");
     // -------------------------------------------------------------- softmax
-    const int tt = (warp - 4) >> 2;               // query tile of this warpgroup
-    const int quad = warp & 3;                    // TMEM lane quadrant
-    const int r = quad * 32 + lane;               // row within the tile
+    constexpr int kFh = D / 2;                     // accumulator columns kept in registers
+    const int tt = (warp - 8) >> 2;                // query tile of this warpgroup
+    const int quad = warp & 3;                     // TMEM lane quadrant
+    const int r = quad * 32 + lane;                // row within the tile
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
     const uint32_t tA = tbase + tt * 256 + 128 + lane_off;
+    float4* Fs = reinterpret_cast<float4*>(smem + C::oF) + (tt * kRows + r) * (C::kFRow / 4);
     const float kLog2e = 1.4426950408889634f;
     uint32_t g = 0;
     bool ok = true;
-    float F[D];
+    float F[kFh];
+    // F += w * (integer accumulator), then reset the accumulator.  The first
+    // half of the columns is in registers, the second half in shared memory.
+    auto fold = [&](float w, int dump_t, bool dump_now) {
+#pragma unroll
+      for (int c = 0; c < D; c += 32) {
+        uint32_t a[32];
+        tmem_ld32(tA + c, a);
+        if (c < kFh) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            F[c + i] = fmaf(w, __int_as_float(static_cast<int>(a[i])) - kMagicF, F[c + i]);
+        } else {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            float4 f = Fs[(c - kFh) / 4 + q];
+            f.x = fmaf(w, __int_as_float(static_cast<int>(a[4 * q + 0])) - kMagicF, f.x);
+            f.y = fmaf(w, __int_as_float(static_cast<int>(a[4 * q + 1])) - kMagicF, f.y);
+            f.z = fmaf(w, __int_as_float(static_cast<int>(a[4 * q + 2])) - kMagicF, f.z);
+            f.w = fmaf(w, __int_as_float(static_cast<int>(a[4 * q + 3])) - kMagicF, f.w);
+            Fs[(c - kFh) / 4 + q] = f;
+          }
+        }
+        if (DUMP && dump_now && prm.dump_acc) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            prm.dump_acc[(static_cast<size_t>(r) * nb + dump_t) * D + wide_to_dim(c + i)] =
+                (static_cast<int>(a[i]) - static_cast<int>(kMagic)) / 16;
+        }
+        tmem_fill32(tA + c, kMagic);
+      }
+    };
     for (int item = blockIdx.x; item < prm.nitems && ok; item += gridDim.x) {
       const int bh = item / prm.npairs, pair = item % prm.npairs;
       const int qtile = pair * 2 + tt;
@@ -355,7 +398,9 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       const float cpi = __fmul_rn(ci, kLog2e);
       const bool dump_tile = DUMP && bh == prm.dump_bh && qtile == prm.dump_tile && row_ok;
 #pragma unroll
-      for (int i = 0; i < D; ++i) F[i] = 0.0f;
+      for (int i = 0; i < kFh; ++i) F[i] = 0.0f;
+#pragma unroll
+      for (int q = 0; q < kFh / 4; ++q) Fs[q] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
       float m_run = -INFINITY, m_ref = 0.0f, w = 1.0f, Lf = 0.0f;
       int Lrun = 0;
       // fresh integer accumulator
@@ -367,82 +412,87 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (!(ok = wait_at(B.s_full + tt * 2 + buf, (g >> 1) & 1, abort_flag, 10u, g))) break;
         __syncwarp();
         tc_fence_after();
-        uint32_t raw[BN];
-        tmem_ld<BN>(tS, raw);
         const int ks = g % C::kKS;
         if (!(ok = wait_at(B.kw_full + ks, (g / C::kKS) & 1, abort_flag, 11u, g))) break;
         const float* ksc = reinterpret_cast<const float*>(smem + C::oKsc) + ks * BN;
         const int nvalid = min(BN, prm.N - t * BN);
-        float v[BN];
+        constexpr int kCh = BN < 32 ? BN : 32;  // columns per TMEM access
+        // Pass 1: v = S_int * s_k exactly (256 S_int is exact in fp32 and s_k/256
+        // a power-of-two scaling), written back over S; block maximum.  Keys
+        // past N give NaN, which fmaxf skips.
+        float vmax = -INFINITY;
 #pragma unroll
-        for (int j = 0; j < BN; ++j) {
-          const float f = __int_as_float(static_cast<int>(raw[j]) + static_cast<int>(kMagic)) - kMagicF;
-          v[j] = f * ksc[j];
+        for (int c0 = 0; c0 < BN; c0 += kCh) {
+          uint32_t raw[kCh];
+          tmem_ld<kCh>(tS + c0, raw);
+          if (dump_tile) {
+            for (int j = 0; j < kCh && c0 + j < nvalid; ++j)
+              if (prm.dump_s) prm.dump_s[static_cast<size_t>(r) * prm.N + t * BN + c0 + j] = static_cast<int32_t>(raw[j]) / 256;
+          }
+#pragma unroll
+          for (int j = 0; j < kCh; j += 4) {
+            const float4 sc = *reinterpret_cast<const float4*>(ksc + c0 + j);
+            raw[j + 0] = __float_as_uint(static_cast<float>(static_cast<int>(raw[j + 0])) * sc.x);
+            raw[j + 1] = __float_as_uint(static_cast<float>(static_cast<int>(raw[j + 1])) * sc.y);
+            raw[j + 2] = __float_as_uint(static_cast<float>(static_cast<int>(raw[j + 2])) * sc.z);
+            raw[j + 3] = __float_as_uint(static_cast<float>(static_cast<int>(raw[j + 3])) * sc.w);
+          }
+#pragma unroll
+          for (int j = 0; j + 1 < kCh; j += 2) vmax = max3(vmax, __uint_as_float(raw[j]), __uint_as_float(raw[j + 1]));
+          if constexpr (kCh == 32) tmem_st32(tS + c0, raw);
+          else tmem_st16(tS + c0, raw);
         }
-        if (nvalid < BN) {
-#pragma unroll
-          for (int j = 0; j < BN; ++j)
-            if (j >= nvalid) v[j] = -INFINITY;
-        }
-        float vmax = v[0];
-#pragma unroll
-        for (int j = 1; j + 1 < BN; j += 2) vmax = max3(vmax, v[j], v[j + 1]);
-        if (BN % 2 == 0) vmax = fmaxf(vmax, v[BN - 1]);
         const float m_blk = __fmul_rn(vmax, ci);
         const float m_new = fmaxf(m_run, m_blk);
         const bool grow = m_new > m_run;
         const float Mp = __fmul_rn(m_new, kLog2e);
+        // Pass 2: P code c + 8 = rint(15 exp2(y)): adding 15 e to 1.5 * 2^23
+        // rounds it to an integer that lands in the low byte of the sum's bits.
         uint32_t words[C::kKeysPV / 4];
+#pragma unroll
+        for (int c0 = 0; c0 < BN; c0 += kCh) {
+          uint32_t vb[kCh];
+          tmem_ld<kCh>(tS + c0, vb);
+#pragma unroll
+          for (int q = 0; q < kCh / 4; ++q) {
+            uint32_t tb[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float pe = ex2_approx(fmaf(__uint_as_float(vb[4 * q + e]), cpi, -Mp));
+              tb[e] = __float_as_uint(fmaf(15.0f, pe, kMagicF));
+            }
+            words[c0 / 4 + q] = __byte_perm(__byte_perm(tb[0], tb[1], 0x0040), __byte_perm(tb[2], tb[3], 0x0040), 0x5410);
+          }
+        }
+        if (nvalid < BN) {  // last, ragged block: codes of keys past N are 0
+#pragma unroll
+          for (int q = 0; q < BN / 4; ++q) {
+            const int lim = nvalid - 4 * q;
+            words[q] &= lim >= 4 ? 0xFFFFFFFFu : (lim <= 0 ? 0u : (0xFFFFFFFFu >> (8 * (4 - lim))));
+          }
+        }
         int lq = 0;
 #pragma unroll
-        for (int q = 0; q < BN / 4; ++q) {
-          uint32_t tb[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int j = 4 * q + e;
-            float y = fmaf(v[j], cpi, -Mp);
-            if (nvalid < BN && j >= nvalid) y = -INFINITY;
-            const float pe = ex2_approx(y);
-            tb[e] = __float_as_uint(fmaf(15.0f, pe, kMagicF));
-          }
-          const uint32_t wd = __byte_perm(__byte_perm(tb[0], tb[1], 0x0040), __byte_perm(tb[2], tb[3], 0x0040), 0x5410);
-          words[q] = wd;
-          lq = __dp4a(static_cast<int>(wd), 0x01010101, lq);
-        }
+        for (int q = 0; q < BN / 4; ++q) lq = __dp4a(static_cast<int>(words[q]), 0x01010101, lq);
 #pragma unroll
         for (int q = BN / 4; q < C::kKeysPV / 4; ++q) words[q] = 0u;
         if constexpr (C::kKeysPV / 4 == 16) tmem_st16(tS, words);
         else if constexpr (C::kKeysPV / 4 == 8) tmem_st8(tS, words);
-        if (dump_tile) {
-          for (int j = 0; j < nvalid; ++j) {
-            const size_t o = static_cast<size_t>(r) * prm.N + t * BN + j;
-            if (prm.dump_s) prm.dump_s[o] = static_cast<int32_t>(raw[j]) / 256;
-            if (prm.dump_p) prm.dump_p[o] = static_cast<int8_t>(((words[j >> 2] >> (8 * (j & 3))) & 0xFF) - 8);
-          }
+        if (dump_tile && prm.dump_p) {
+          for (int j = 0; j < nvalid; ++j)
+            prm.dump_p[static_cast<size_t>(r) * prm.N + t * BN + j] =
+                static_cast<int8_t>(((words[j >> 2] >> (8 * (j & 3))) & 0xFF) - 8);
         }
         // Fold the integer accumulator into F when a row's maximum grows (its
-        // earlier codes used the old maximum) or its magnitude bound is near
-        // the exact range of the read-back (|acc| < 2^22).
+        // earlier codes used the old maximum) or its magnitude bound nears the
+        // exact range of the read-back (|acc| < 2^22).
         const bool near_bound = (Lrun + 15 * BN) * 112 >= (1 << 22) - 4096;
         const bool need = (t > 0) && (grow || near_bound || DUMP);
         if (__any_sync(0xFFFFFFFFu, need)) {
           if (!(ok = wait_at(B.pv_done + tt * 2 + ((g - 1) & 1), ((g - 1) >> 1) & 1, abort_flag, 12u, g))) break;
           __syncwarp();
           tc_fence_after();
-#pragma unroll
-          for (int c = 0; c < D; c += 32) {
-            uint32_t a[32];
-            tmem_ld32(tA + c, a);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const float af = __int_as_float(static_cast<int>(a[i])) - kMagicF;
-              F[c + i] = fmaf(w, af, F[c + i]);
-              if (dump_tile && prm.dump_acc)
-                prm.dump_acc[(static_cast<size_t>(r) * nb + (t - 1)) * D + wide_to_dim(c + i)] =
-                    (static_cast<int>(a[i]) - static_cast<int>(kMagic)) / 16;
-            }
-            tmem_fill32(tA + c, kMagic);
-          }
+          fold(w, t - 1, dump_tile);
           Lf = fmaf(w, static_cast<float>(Lrun), Lf);
           Lrun = 0;
         }
@@ -454,7 +504,11 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           if (x > 64.0f) {
             const float sc = ex2_approx(-x);
 #pragma unroll
-            for (int i = 0; i < D; ++i) F[i] *= sc;
+            for (int i = 0; i < kFh; ++i) F[i] *= sc;
+            for (int q = 0; q < kFh / 4; ++q) {
+              float4 f = Fs[q];
+              Fs[q] = make_float4(f.x * sc, f.y * sc, f.z * sc, f.w * sc);
+            }
             Lf *= sc;
             m_ref = m_new;
             w = 1.0f;
@@ -476,23 +530,12 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       if (!(ok = wait_at(B.pv_done + tt * 2 + ((g - 1) & 1), ((g - 1) >> 1) & 1, abort_flag, 13u, g))) break;
       __syncwarp();
       tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < D; c += 32) {
-        uint32_t a[32];
-        tmem_ld32(tA + c, a);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float af = __int_as_float(static_cast<int>(a[i])) - kMagicF;
-          F[c + i] = fmaf(w, af, F[c + i]);
-          if (dump_tile && prm.dump_acc)
-            prm.dump_acc[(static_cast<size_t>(r) * nb + (nb - 1)) * D + wide_to_dim(c + i)] =
-                (static_cast<int>(a[i]) - static_cast<int>(kMagic)) / 16;
-        }
-      }
+      fold(w, nb - 1, dump_tile);
       Lf = fmaf(w, static_cast<float>(Lrun), Lf);
       if (row_ok) {
         const float inv = 1.0f / (16.0f * Lf);
         const float* sv = prm.sv + static_cast<size_t>(bh) * D;
+        const float* Fsf = reinterpret_cast<const float*>(Fs);
         __nv_bfloat16* orow = prm.out + (static_cast<size_t>(bh) * prm.N + row) * D;
 #pragma unroll
         for (int c = 0; c < D; c += 32) {
@@ -502,9 +545,9 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
               const int d = c + 8 * a + 2 * b;
-              const float o0 = F[c + 4 * a + b] * __ldg(sv + d) * inv;
-              const float o1 = F[c + 16 + 4 * a + b] * __ldg(sv + d + 1) * inv;
-              const __nv_bfloat162 h = __floats2bfloat162_rn(o0, o1);
+              const float f0 = c < kFh ? F[c + 4 * a + b] : Fsf[c - kFh + 4 * a + b];
+              const float f1 = c < kFh ? F[c + 16 + 4 * a + b] : Fsf[c - kFh + 16 + 4 * a + b];
+              const __nv_bfloat162 h = __floats2bfloat162_rn(f0 * __ldg(sv + d) * inv, f1 * __ldg(sv + d + 1) * inv);
               pk[4 * a + b] = *reinterpret_cast<const uint32_t*>(&h);
             }
           uint4* dst = reinterpret_cast<uint4*>(orow + c);

@@ -16,9 +16,11 @@ namespace ra {
 constexpr uint32_t kStatusBadPosition = 1u;
 constexpr uint32_t kStatusTimeout = 2u;
 
-// Bound on every spin-wait: 2^22 polls with back-off (a few seconds at most),
-// far above any legitimate wait, so a wait that never completes ends with an
-// error status instead of a hang.
+// Bound on every mbarrier wait: 2 s of wall time (%globaltimer), far above any
+// legitimate wait, so a wait that never completes ends with an error status
+// instead of a hang.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// Iteration bound for the few waits that poll without a time source.
 constexpr uint32_t kSpinLimit = 1u << 22;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -54,20 +56,47 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
 // Waits for the phase with the given parity to complete.  Returns 1 when it
 // completed, 0 when another thread raised *abort, and -1 when this wait ran
-// past kSpinLimit (it then raises *abort itself).
-__device__ __forceinline__ int mbar_wait_ex(uint64_t* bar, uint32_t parity, volatile int* abort) {
-  if (mbar_try_wait(bar, parity)) return 1;
-  for (uint32_t it = 0; it < kSpinLimit; ++it) {
-    if (mbar_try_wait(bar, parity)) return 1;
-    if ((it & 255u) == 255u) {
+// past kWaitLimitNs (it then raises *abort itself).  Between non-blocking tests
+// the thread sleeps, starting at 16 ns and doubling up to max_sleep_ns: short
+// waits end promptly, long waits poll rarely and leave issue slots to the warps
+// doing the arithmetic.  The abort flag and the clock are read every 32nd test
+// only, to keep each test cheap.
+__device__ __forceinline__ int mbar_wait_ex(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                            uint32_t max_sleep_ns = 64) {
+  if (mbar_test_wait(bar, parity)) return 1;
+  const uint64_t t0 = global_ns();
+  uint32_t sleep = 16;
+  for (uint32_t n = 1;; ++n) {
+    __nanosleep(sleep);
+    if (mbar_test_wait(bar, parity)) return 1;
+    sleep = min(sleep * 2, max_sleep_ns);
+    if ((n & 31u) == 0) {
       if (*abort) return 0;
-      __nanosleep(64);
+      if (global_ns() - t0 > kWaitLimitNs) {
+        *abort = 1;
+        return -1;
+      }
     }
   }
-  *abort = 1;
-  return -1;
 }
 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
@@ -168,6 +197,18 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
       "tcgen05.wait::st.sync.aligned;"
       ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
         "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n\t"
+      "tcgen05.wait::st.sync.aligned;"
+      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+        "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+        "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
 }
 
