@@ -104,30 +104,33 @@ def _config(wl, extra=None):
     return c
 
 
-def cpu_baseline(wl, target_s: float = 15.0):
+def cpu_baseline(wl, target_s: float = 15.0, x=None):
     """The oracle, as it stands, on a bounded sample of the workload: the
     prologue of head 0 and the attention of as many 128-row query tiles of head 0
-    as fit in about target_s seconds; value prorated to the metric's unit."""
-    import numpy as np
+    as fit in about target_s seconds (tiles visited in a strided order so the
+    sample spans the sequence); value prorated to the metric's unit."""
     import oracle
     from synth import inputs as si
-    x = si.make_inputs(wl, heads=(0,))
+    if x is None:
+        x = si.make_inputs(wl, heads=(0,))
     p = oracle.problem(wl)
     t0 = time.perf_counter()
     h = oracle.prologue_head(p, x["q"][0, 0], x["k"][0, 0], x["v"][0, 0], x["pos"])
     t_pro = time.perf_counter() - t0
+    ntiles = -(-wl.N // 128)
+    stride = max(1, ntiles // 16)
+    order = [t for off in range(stride) for t in range(off, ntiles, stride)]
     rows = 0
     t_att = 0.0
-    ntiles = -(-wl.N // 128)
-    tile = 0
-    while t_att < target_s and tile < ntiles:
+    for tile in order:
+        if t_att >= target_s:
+            break
         r0 = tile * 128
         r1 = min(r0 + 128, wl.N)
         t0 = time.perf_counter()
         oracle.attention_int4_rows(p, h, r0, r1)
         t_att += time.perf_counter() - t0
         rows += r1 - r0
-        tile += max(1, ntiles // 16)
     t = t_att + t_pro * rows / wl.N
     ops = 4.0 * rows * wl.N * wl.D
     return {"value": ops / t / 1e12, "unit": "TOPS", "cores": oracle.num_threads(), "kind": "oracle",
@@ -275,10 +278,14 @@ def run_reference(args):
     wl = _workload(args.workload)
     import oracle
     oracle.lib()
+    from synth import inputs as si
+    x = si.make_inputs(wl, heads=(0,))
+    # each step is one bounded sample; the whole run stays within a few minutes
+    per_step = max(1.0, min(args.ref_seconds, 180.0 / max(1, args.warmup + args.steps)))
     vals = []
     base = None
     for i in range(args.warmup + args.steps):
-        r = cpu_baseline(wl, target_s=args.ref_seconds)
+        r = cpu_baseline(wl, target_s=per_step, x=x)
         if i >= args.warmup:
             vals.append(r["value"])
             base = r
