@@ -133,12 +133,46 @@ __device__ __forceinline__ void widen_tile(const uint8_t* pk, uint8_t* wide, int
   }
 }
 
+// Per-thread chunk offsets of widen_tile for a fixed tile height, computed
+// once: every K/V block has the same layout, so the widening warps only load,
+// widen and store in their loop.
+template <int D, int ROWS>
+struct WidenPlan {
+  static constexpr int kChunks = ROWS * (D / 32);
+  static constexpr int kIter = (kChunks + 127) / 128;
+  uint32_t src[kIter], lo[kIter], hi[kIter];
+  __device__ __forceinline__ void init(int tid) {
+#pragma unroll
+    for (int k = 0; k < kIter; ++k) {
+      const int idx = tid + 128 * k;
+      const int r = idx / (D / 32), pc = idx % (D / 32);
+      src[k] = idx < kChunks ? static_cast<uint32_t>(r * (D / 2) + pc * 16) : ~0u;
+      lo[k] = swz_offset(r, 2 * pc, D);
+      hi[k] = swz_offset(r, 2 * pc + 1, D);
+    }
+  }
+  __device__ __forceinline__ void run(const uint8_t* pk, uint8_t* wide) const {
+#pragma unroll
+    for (int k = 0; k < kIter; ++k)
+      if (kChunks % 128 == 0 || src[k] != ~0u) widen_chunk(pk + src[k], wide + lo[k], wide + hi[k]);
+  }
+};
+
 // Widened position n (0..D-1) of a row -> channel.
 __host__ __device__ constexpr int wide_to_dim(int n) {
   return (n & ~31) + 8 * ((n & 15) >> 2) + 2 * (n & 3) + ((n >> 4) & 1);
 }
 
 __device__ __forceinline__ float max3(float a, float b, float c) { return fmaxf(a, fmaxf(b, c)); }
+
+// Maximum of n values as a tree of 3-way maxima (short dependency chains).
+template <int n>
+__device__ __forceinline__ float tree_max(const float* x) {
+  if constexpr (n == 1) return x[0];
+  else if constexpr (n == 2) return fmaxf(x[0], x[1]);
+  else if constexpr (n == 3) return max3(x[0], x[1], x[2]);
+  else return max3(tree_max<n / 3>(x), tree_max<n / 3>(x + n / 3), tree_max<n - 2 * (n / 3)>(x + 2 * (n / 3)));
+}
 
 __device__ __forceinline__ void set_status(uint32_t bits) { atomicOr(&g_attn_status, bits); }
 
@@ -307,6 +341,8 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     } else if (warp >= 4) {
       // ------------------------------------------------------------ widening warps
       const int wt = threadIdx.x - 128;  // 0..127
+      WidenPlan<D, BN> plan;
+      plan.init(wt);
       uint32_t g = 0, li = 0;
       bool ok = true;
       for (int item = blockIdx.x; item < prm.nitems && ok; item += gridDim.x, ++li) {
@@ -323,7 +359,7 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           if (!(ok = wait_at(B.pk_full + s, (g / C::kPS) & 1, abort_flag, 9u, g, 128u))) break;
           if (!(ok = wait_at(B.kw_empty + ks, ((g / C::kKS) & 1) ^ 1, abort_flag, 15u, g, 256u))) break;
           const uint8_t* pk = smem + C::oPk + s * 2 * C::kPkHalf;
-          widen_tile<D>(pk, smem + C::oKw + ks * C::kKwStride, BN, wt, 128);
+          plan.run(pk, smem + C::oKw + ks * C::kKwStride);
           if (wt < BN) {
             const int j = t * BN + wt;
             float* ksc = reinterpret_cast<float*>(smem + C::oKsc) + ks * BN;
@@ -336,7 +372,7 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           __syncwarp();
           if (lane == 0) mbar_arrive(B.kw_full + ks);
           if (!(ok = wait_at(B.vw_empty + vs, ((g / C::kVS) & 1) ^ 1, abort_flag, 16u, g, 256u))) break;
-          widen_tile<D>(pk + C::kPkHalf, smem + C::oVw + vs * C::kVwStride, BN, wt, 128);
+          plan.run(pk + C::kPkHalf, smem + C::oVw + vs * C::kVwStride);
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) { mbar_arrive(B.vw_full + vs); mbar_arrive(B.pk_empty + s); }
@@ -355,29 +391,39 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const uint32_t tA = tbase + tt * 256 + 128 + lane_off;
     float4* Fs = reinterpret_cast<float4*>(smem + C::oF) + (tt * kRows + r) * (C::kFRow / 4);
     const float kLog2e = 1.4426950408889634f;
+    // Arithmetic on pairs of fp32 (sm_100 f32x2 instructions: two lanes per
+    // instruction, each rounded exactly like the scalar form).
+    const float2 kNegMagic2 = make_float2(-kMagicF, -kMagicF);
+    const float2 kMagic2 = make_float2(kMagicF, kMagicF);
+    const float2 k15x2 = make_float2(15.0f, 15.0f);
     uint32_t g = 0;
     bool ok = true;
-    float F[kFh];
+    float2 F2[kFh / 2];  // F[2i], F[2i+1]
     // F += w * (integer accumulator), then reset the accumulator.  The first
     // half of the columns is in registers, the second half in shared memory.
     auto fold = [&](float w, int dump_t, bool dump_now) {
+      const float2 w2 = make_float2(w, w);
 #pragma unroll
       for (int c = 0; c < D; c += 32) {
         uint32_t a[32];
         tmem_ld32(tA + c, a);
         if (c < kFh) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i)
-            F[c + i] = fmaf(w, __int_as_float(static_cast<int>(a[i])) - kMagicF, F[c + i]);
+          for (int i = 0; i < 16; ++i)
+            F2[c / 2 + i] = __ffma2_rn(
+                w2, __fadd2_rn(make_float2(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1])), kNegMagic2),
+                F2[c / 2 + i]);
         } else {
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
-            float4 f = Fs[(c - kFh) / 4 + q];
-            f.x = fmaf(w, __int_as_float(static_cast<int>(a[4 * q + 0])) - kMagicF, f.x);
-            f.y = fmaf(w, __int_as_float(static_cast<int>(a[4 * q + 1])) - kMagicF, f.y);
-            f.z = fmaf(w, __int_as_float(static_cast<int>(a[4 * q + 2])) - kMagicF, f.z);
-            f.w = fmaf(w, __int_as_float(static_cast<int>(a[4 * q + 3])) - kMagicF, f.w);
-            Fs[(c - kFh) / 4 + q] = f;
+            const float4 f = Fs[(c - kFh) / 4 + q];
+            const float2 lo = __ffma2_rn(
+                w2, __fadd2_rn(make_float2(__uint_as_float(a[4 * q + 0]), __uint_as_float(a[4 * q + 1])), kNegMagic2),
+                make_float2(f.x, f.y));
+            const float2 hi = __ffma2_rn(
+                w2, __fadd2_rn(make_float2(__uint_as_float(a[4 * q + 2]), __uint_as_float(a[4 * q + 3])), kNegMagic2),
+                make_float2(f.z, f.w));
+            Fs[(c - kFh) / 4 + q] = make_float4(lo.x, lo.y, hi.x, hi.y);
           }
         }
         if (DUMP && dump_now && prm.dump_acc) {
@@ -396,9 +442,10 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       const bool row_ok = row < prm.N;
       const float ci = row_ok ? __fmul_rn(prm.sq[static_cast<size_t>(bh) * prm.N + row], prm.inv_sqrt_d) : 0.0f;
       const float cpi = __fmul_rn(ci, kLog2e);
+      const float2 cpi2 = make_float2(cpi, cpi);
       const bool dump_tile = DUMP && bh == prm.dump_bh && qtile == prm.dump_tile && row_ok;
 #pragma unroll
-      for (int i = 0; i < kFh; ++i) F[i] = 0.0f;
+      for (int i = 0; i < kFh / 2; ++i) F2[i] = make_float2(0.0f, 0.0f);
 #pragma unroll
       for (int q = 0; q < kFh / 4; ++q) Fs[q] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
       float m_run = -INFINITY, m_ref = 0.0f, w = 1.0f, Lf = 0.0f;
@@ -414,55 +461,45 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tc_fence_after();
         const int ks = g % C::kKS;
         if (!(ok = wait_at(B.kw_full + ks, (g / C::kKS) & 1, abort_flag, 11u, g))) break;
-        const float* ksc = reinterpret_cast<const float*>(smem + C::oKsc) + ks * BN;
+        const float4* ksc = reinterpret_cast<const float4*>(smem + C::oKsc) + ks * (BN / 4);
         const int nvalid = min(BN, prm.N - t * BN);
-        constexpr int kCh = BN < 32 ? BN : 32;  // columns per TMEM access
-        // Pass 1: v = S_int * s_k exactly (256 S_int is exact in fp32 and s_k/256
-        // a power-of-two scaling), written back over S; block maximum.  Keys
-        // past N give NaN, which fmaxf skips.
-        float vmax = -INFINITY;
-#pragma unroll
-        for (int c0 = 0; c0 < BN; c0 += kCh) {
-          uint32_t raw[kCh];
-          tmem_ld<kCh>(tS + c0, raw);
-          if (dump_tile) {
-            for (int j = 0; j < kCh && c0 + j < nvalid; ++j)
-              if (prm.dump_s) prm.dump_s[static_cast<size_t>(r) * prm.N + t * BN + c0 + j] = static_cast<int32_t>(raw[j]) / 256;
-          }
-#pragma unroll
-          for (int j = 0; j < kCh; j += 4) {
-            const float4 sc = *reinterpret_cast<const float4*>(ksc + c0 + j);
-            raw[j + 0] = __float_as_uint(static_cast<float>(static_cast<int>(raw[j + 0])) * sc.x);
-            raw[j + 1] = __float_as_uint(static_cast<float>(static_cast<int>(raw[j + 1])) * sc.y);
-            raw[j + 2] = __float_as_uint(static_cast<float>(static_cast<int>(raw[j + 2])) * sc.z);
-            raw[j + 3] = __float_as_uint(static_cast<float>(static_cast<int>(raw[j + 3])) * sc.w);
-          }
-#pragma unroll
-          for (int j = 0; j + 1 < kCh; j += 2) vmax = max3(vmax, __uint_as_float(raw[j]), __uint_as_float(raw[j + 1]));
-          if constexpr (kCh == 32) tmem_st32(tS + c0, raw);
-          else tmem_st16(tS + c0, raw);
+        // v = S_int * s_k for the whole block, in registers (256 S_int is exact
+        // in fp32 and s_k/256 a power-of-two scaling, so v is S_int * s_k
+        // rounded once).  Keys past N give NaN, which fmaxf skips.
+        uint32_t raw[BN];
+        tmem_ld<BN>(tS, raw);
+        if (dump_tile) {
+          for (int j = 0; j < nvalid; ++j)
+            if (prm.dump_s) prm.dump_s[static_cast<size_t>(r) * prm.N + t * BN + j] = static_cast<int32_t>(raw[j]) / 256;
         }
+        float2 v2[BN / 2];
+#pragma unroll
+        for (int j = 0; j < BN; j += 4) {
+          const float4 sc = ksc[j / 4];
+          v2[j / 2] = __fmul2_rn(make_float2(static_cast<float>(static_cast<int>(raw[j])),
+                                             static_cast<float>(static_cast<int>(raw[j + 1]))),
+                                 make_float2(sc.x, sc.y));
+          v2[j / 2 + 1] = __fmul2_rn(make_float2(static_cast<float>(static_cast<int>(raw[j + 2])),
+                                                 static_cast<float>(static_cast<int>(raw[j + 3]))),
+                                     make_float2(sc.z, sc.w));
+        }
+        const float vmax = tree_max<BN>(reinterpret_cast<const float*>(v2));
         const float m_blk = __fmul_rn(vmax, ci);
         const float m_new = fmaxf(m_run, m_blk);
         const bool grow = m_new > m_run;
         const float Mp = __fmul_rn(m_new, kLog2e);
-        // Pass 2: P code c + 8 = rint(15 exp2(y)): adding 15 e to 1.5 * 2^23
-        // rounds it to an integer that lands in the low byte of the sum's bits.
+        const float2 nMp2 = make_float2(-Mp, -Mp);
+        // P code c + 8 = rint(15 exp2(y)): adding 15 e to 1.5 * 2^23 rounds it
+        // to an integer that lands in the low byte of the sum's bits.
         uint32_t words[C::kKeysPV / 4];
 #pragma unroll
-        for (int c0 = 0; c0 < BN; c0 += kCh) {
-          uint32_t vb[kCh];
-          tmem_ld<kCh>(tS + c0, vb);
-#pragma unroll
-          for (int q = 0; q < kCh / 4; ++q) {
-            uint32_t tb[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float pe = ex2_approx(fmaf(__uint_as_float(vb[4 * q + e]), cpi, -Mp));
-              tb[e] = __float_as_uint(fmaf(15.0f, pe, kMagicF));
-            }
-            words[c0 / 4 + q] = __byte_perm(__byte_perm(tb[0], tb[1], 0x0040), __byte_perm(tb[2], tb[3], 0x0040), 0x5410);
-          }
+        for (int q = 0; q < BN / 4; ++q) {
+          const float2 x01 = __ffma2_rn(v2[2 * q], cpi2, nMp2);
+          const float2 x23 = __ffma2_rn(v2[2 * q + 1], cpi2, nMp2);
+          const float2 t01 = __ffma2_rn(k15x2, make_float2(ex2_approx(x01.x), ex2_approx(x01.y)), kMagic2);
+          const float2 t23 = __ffma2_rn(k15x2, make_float2(ex2_approx(x23.x), ex2_approx(x23.y)), kMagic2);
+          words[q] = __byte_perm(__byte_perm(__float_as_uint(t01.x), __float_as_uint(t01.y), 0x0040),
+                                 __byte_perm(__float_as_uint(t23.x), __float_as_uint(t23.y), 0x0040), 0x5410);
         }
         if (nvalid < BN) {  // last, ragged block: codes of keys past N are 0
 #pragma unroll
@@ -471,9 +508,12 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             words[q] &= lim >= 4 ? 0xFFFFFFFFu : (lim <= 0 ? 0u : (0xFFFFFFFFu >> (8 * (4 - lim))));
           }
         }
-        int lq = 0;
+        // Sum of the row's codes (+8 each): bytes are at most 15, so plain
+        // word additions of up to 16 words cannot carry between bytes.
+        uint32_t wsum = 0;
 #pragma unroll
-        for (int q = 0; q < BN / 4; ++q) lq = __dp4a(static_cast<int>(words[q]), 0x01010101, lq);
+        for (int q = 0; q < BN / 4; ++q) wsum += words[q];
+        const int lq = static_cast<int>(__dp4a(wsum, 0x01010101u, 0u));  // unsigned bytes (up to 240)
 #pragma unroll
         for (int q = BN / 4; q < C::kKeysPV / 4; ++q) words[q] = 0u;
         if constexpr (C::kKeysPV / 4 == 16) tmem_st16(tS, words);
@@ -503,8 +543,9 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           const float x = __fmul_rn(m_new - m_ref, kLog2e);
           if (x > 64.0f) {
             const float sc = ex2_approx(-x);
+            const float2 sc2 = make_float2(sc, sc);
 #pragma unroll
-            for (int i = 0; i < kFh; ++i) F[i] *= sc;
+            for (int i = 0; i < kFh / 2; ++i) F2[i] = __fmul2_rn(F2[i], sc2);
             for (int q = 0; q < kFh / 4; ++q) {
               float4 f = Fs[q];
               Fs[q] = make_float4(f.x * sc, f.y * sc, f.z * sc, f.w * sc);
@@ -537,6 +578,7 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const float* sv = prm.sv + static_cast<size_t>(bh) * D;
         const float* Fsf = reinterpret_cast<const float*>(Fs);
         __nv_bfloat16* orow = prm.out + (static_cast<size_t>(bh) * prm.N + row) * D;
+        auto fget = [&](int i) -> float { return (i & 1) ? F2[i >> 1].y : F2[i >> 1].x; };
 #pragma unroll
         for (int c = 0; c < D; c += 32) {
           uint32_t pk[16];
@@ -545,8 +587,8 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
               const int d = c + 8 * a + 2 * b;
-              const float f0 = c < kFh ? F[c + 4 * a + b] : Fsf[c - kFh + 4 * a + b];
-              const float f1 = c < kFh ? F[c + 16 + 4 * a + b] : Fsf[c - kFh + 16 + 4 * a + b];
+              const float f0 = c < kFh ? fget(c + 4 * a + b) : Fsf[c - kFh + 4 * a + b];
+              const float f1 = c < kFh ? fget(c + 16 + 4 * a + b) : Fsf[c - kFh + 16 + 4 * a + b];
               const __nv_bfloat162 h = __floats2bfloat162_rn(f0 * __ldg(sv + d) * inv, f1 * __ldg(sv + d + 1) * inv);
               pk[4 * a + b] = *reinterpret_cast<const uint32_t*>(&h);
             }
