@@ -399,10 +399,17 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     uint32_t g = 0;
     bool ok = true;
     float2 F2[kFh / 2];  // F[2i], F[2i+1]
-    // F += w * (integer accumulator), then reset the accumulator.  The first
-    // half of the columns is in registers, the second half in shared memory.
-    auto fold = [&](float w, int dump_t, bool dump_now) {
-      const float2 w2 = make_float2(w, w);
+    // F += coef * (integer accumulator A); with reset, A is then set back to
+    // zero (its bits to 1.5 * 2^23).  The first half of the columns of F is in
+    // registers, the second half in shared memory.
+    //
+    // Without reset, A keeps accumulating across a change of the row maximum:
+    // with segments s_k of P.V results between changes, A_k = s_1 + ... + s_k
+    // and segment weights w_k, sum_k w_k s_k = sum_k (w_k - w_(k+1)) A_k plus
+    // w_last A_last, so each change adds (w_old - w_new) A to F and the final
+    // fold adds w_last A.  This needs no TMEM store at a change.
+    auto fold = [&](float coef, bool reset, int dump_t, bool dump_now) {
+      const float2 w2 = make_float2(coef, coef);
 #pragma unroll
       for (int c = 0; c < D; c += 32) {
         uint32_t a[32];
@@ -432,7 +439,7 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             prm.dump_acc[(static_cast<size_t>(r) * nb + dump_t) * D + wide_to_dim(c + i)] =
                 (static_cast<int>(a[i]) - static_cast<int>(kMagic)) / 16;
         }
-        tmem_fill32(tA + c, kMagic);
+        if (reset) tmem_fill32(tA + c, kMagic);
       }
     };
     for (int item = blockIdx.x; item < prm.nitems && ok; item += gridDim.x) {
@@ -449,7 +456,8 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
       for (int q = 0; q < kFh / 4; ++q) Fs[q] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
       float m_run = -INFINITY, m_ref = 0.0f, w = 1.0f, Lf = 0.0f;
-      int Lrun = 0;
+      int Lrun = 0;   // code sum since the last fold (denominator)
+      int Labs = 0;   // code sum since the last reset of A (magnitude bound)
       // fresh integer accumulator
 #pragma unroll
       for (int c = 0; c < D; c += 32) tmem_fill32(tA + c, kMagic);
@@ -526,23 +534,31 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // Fold the integer accumulator into F when a row's maximum grows (its
         // earlier codes used the old maximum) or its magnitude bound nears the
         // exact range of the read-back (|acc| < 2^22).
-        const bool near_bound = (Lrun + 15 * BN) * 112 >= (1 << 22) - 4096;
-        const bool need = (t > 0) && (grow || near_bound || DUMP);
-        if (__any_sync(0xFFFFFFFFu, need)) {
-          if (!(ok = wait_at(B.pv_done + tt * 2 + ((g - 1) & 1), ((g - 1) >> 1) & 1, abort_flag, 12u, g))) break;
-          __syncwarp();
-          tc_fence_after();
-          fold(w, t - 1, dump_tile);
-          Lf = fmaf(w, static_cast<float>(Lrun), Lf);
-          Lrun = 0;
-        }
+        // Weight of the coming segment; a rescale moves the reference max.
+        float w_new = w, sc = 1.0f;
         if (t == 0) {
           m_ref = m_new;
-          w = 1.0f;
+          w_new = 1.0f;
         } else if (grow) {
           const float x = __fmul_rn(m_new - m_ref, kLog2e);
           if (x > 64.0f) {
-            const float sc = ex2_approx(-x);
+            sc = ex2_approx(-x);
+            m_ref = m_new;
+            w_new = 1.0f;
+          } else {
+            w_new = ex2_approx(x);
+          }
+        }
+        // Fold when a row's maximum grows (its earlier codes used the old
+        // maximum); reset A when its magnitude bound nears the exact range of
+        // the read-back (|A| < 2^22).
+        const bool near_bound = (Labs + 15 * BN) * 112 >= (1 << 22) - 4096;
+        const bool reset = __any_sync(0xFFFFFFFFu, (t > 0) && (near_bound || DUMP));
+        if (reset || __any_sync(0xFFFFFFFFu, (t > 0) && grow)) {
+          if (!(ok = wait_at(B.pv_done + tt * 2 + ((g - 1) & 1), ((g - 1) >> 1) & 1, abort_flag, 12u, g))) break;
+          __syncwarp();
+          tc_fence_after();
+          if (sc != 1.0f) {  // new reference maximum: rescale F and the denominator
             const float2 sc2 = make_float2(sc, sc);
 #pragma unroll
             for (int i = 0; i < kFh / 2; ++i) F2[i] = __fmul2_rn(F2[i], sc2);
@@ -551,12 +567,15 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
               Fs[q] = make_float4(f.x * sc, f.y * sc, f.z * sc, f.w * sc);
             }
             Lf *= sc;
-            m_ref = m_new;
-            w = 1.0f;
-          } else {
-            w = ex2_approx(x);
+            w *= sc;
           }
+          fold(reset ? w : w - w_new, reset, t - 1, dump_tile);
+          Lf = fmaf(w, static_cast<float>(Lrun), Lf);
+          Lrun = 0;
+          if (reset) Labs = 0;
         }
+        w = w_new;
+        Labs += lq;
         Lrun += lq;
         m_run = m_new;
         tc_fence_before();
@@ -571,7 +590,7 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       if (!(ok = wait_at(B.pv_done + tt * 2 + ((g - 1) & 1), ((g - 1) >> 1) & 1, abort_flag, 13u, g))) break;
       __syncwarp();
       tc_fence_after();
-      fold(w, nb - 1, dump_tile);
+      fold(w, true, nb - 1, dump_tile);
       Lf = fmaf(w, static_cast<float>(Lrun), Lf);
       if (row_ok) {
         const float inv = 1.0f / (16.0f * Lf);

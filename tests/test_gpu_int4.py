@@ -201,6 +201,22 @@ def test_zero_query_rows_and_zero_value_channels(ra, dev, orc):
     TileCheck(ra, orc, wl, p, codes, host).head(0)
 
 
+def test_uniform_rows_reset_the_integer_accumulator(ra, dev, orc):
+    """A zero query row gives code 15 for every key; over 64 blocks its code
+    sum passes the exact-read-back bound of the integer P.V accumulator, so the
+    kernel folds and resets it mid-row (several times)."""
+    wl = si.WORKLOADS["sweep4096"].with_(H=1)
+    x = si.make_inputs(wl)
+    for a in ("q", "q_bits"):
+        x[a][0, 0, 5] = 0
+        x[a][0, 0, 200] = 0
+    p, codes, host = gu.gpu_forward(ra, wl, x, dev, with_lse=True)
+    chk = TileCheck(ra, orc, wl, p, codes, host)
+    for tile in (0, 1, 31):
+        chk.tile(0, tile)
+    assert chk.end_to_end() <= 1e-3
+
+
 def test_position_outside_grid_is_reported(ra, dev):
     import torch
     wl = si.WORKLOADS["small"].with_(H=1)
