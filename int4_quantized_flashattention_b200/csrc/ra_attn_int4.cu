@@ -24,8 +24,9 @@
 //     accumulator is pre-loaded with the bits of 1.5 * 2^23 so that it reads
 //     back as a float with one subtraction.
 //   * Two 128-row query tiles per CTA share every K/V tile; warp roles:
-//     TMA producer, MMA issuer, two widening warps, two softmax warpgroups
-//     (one thread per query row).  Persistent CTAs, one per SM.
+//     TMA producer, two MMA issuers, four widening warps and 16 softmax warps
+//     (two threads per query row, each with half of the keys of a block and
+//     half of the output columns).  Persistent CTAs, one per SM.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -43,7 +44,7 @@ __device__ uint32_t g_attn_status = 0;
 // First timed-out wait: (site << 24) | (block counter & 0xFFFF) << 8 | (cta & 0xFF).
 __device__ uint32_t g_attn_diag = 0;
 
-constexpr int kThreads = 512;   // 16 warps: see the role map in the kernel
+constexpr int kThreads = 768;   // 24 warps: see the role map in the kernel
 constexpr int kRows = 128;          // query rows per tile = MMA M
 constexpr int kTiles = 2;           // query tiles per CTA
 constexpr uint32_t kMagic = 0x4B400000u;  // bits of 1.5 * 2^23
@@ -66,11 +67,11 @@ struct Cfg {
   static constexpr int oVw = oKw + kKS * ((kKwBytes + 1023) / 1024) * 1024;
   static constexpr int oPk = oVw + kVS * ((kVwBytes + 1023) / 1024) * 1024;
   static constexpr int oKsc = oPk + kPS * 2 * kPkHalf;
-  // Half of every softmax row's fp32 output accumulator lives in shared
-  // memory (the other half in registers); rows padded to avoid bank conflicts.
-  static constexpr int kFRow = D / 2 + 4;                 // floats per row
+  // Half of every softmax thread's fp32 output accumulator columns live in
+  // shared memory (the other half in registers); padded against bank conflicts.
+  static constexpr int kFRow = D / 4 + 4;                 // floats per thread (padded)
   static constexpr int oF = oKsc + kKS * BN * 4;
-  static constexpr int oBar = oF + kTiles * kRows * kFRow * 4;
+  static constexpr int oBar = oF + kTiles * 2 * kRows * kFRow * 4;
   static constexpr int kNumBars = 4 + 2 * kPS + 2 * kKS + 2 * kVS + 4 + 4 + 4 + 2;
   static constexpr int oMisc = oBar + kNumBars * 8;
   static constexpr int kSmem = oMisc + 16 + 1024;       // + alignment slack
@@ -214,9 +215,9 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   if (threadIdx.x == 0) {
     mbar_init(B.qpk_full, 1); mbar_init(B.qpk_empty, 4); mbar_init(B.q_full, 4); mbar_init(B.q_free, 2);
     for (int s = 0; s < C::kPS; ++s) { mbar_init(B.pk_full + s, 1); mbar_init(B.pk_empty + s, 4); }
-    for (int s = 0; s < C::kKS; ++s) { mbar_init(B.kw_full + s, 4); mbar_init(B.kw_empty + s, 2 + 8); }
+    for (int s = 0; s < C::kKS; ++s) { mbar_init(B.kw_full + s, 4); mbar_init(B.kw_empty + s, 2 + 16); }
     for (int s = 0; s < C::kVS; ++s) { mbar_init(B.vw_full + s, 4); mbar_init(B.vw_empty + s, 2); }
-    for (int s = 0; s < 4; ++s) { mbar_init(B.s_full + s, 1); mbar_init(B.p_full + s, 4); mbar_init(B.pv_done + s, 1); }
+    for (int s = 0; s < 4; ++s) { mbar_init(B.s_full + s, 1); mbar_init(B.p_full + s, 8); mbar_init(B.pv_done + s, 1); }
     mbar_init(B.drain, 1);
     mbar_init(B.drain + 1, 1);
     *abort_flag = 0;
@@ -237,7 +238,8 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
   const int nb = prm.nblocks;
   // Roles: warp 0 TMA producer, warp 1 MMA issuer of tile 0 and TMEM owner,
   // warp 2 MMA issuer of tile 1, warp 3 idle, warps 4-7 widen codes (one per
-  // SM sub-partition), warps 8-11 and 12-15 softmax of query tiles 0 and 1.
+  // SM sub-partition), warps 8-15 and 16-23 softmax of query tiles 0 and 1
+  // (two threads per row, 16 rows per warp).
   if (warp < 8) {
     if (warp < 4) asm volatile("setmaxnreg.dec.sync.aligned.u32 56;");
     else asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
@@ -381,15 +383,24 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       if (!ok) set_status(kStatusTimeout);
     }
   } else {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 208;");
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 96;");
     // -------------------------------------------------------------- softmax
-    constexpr int kFh = D / 2;                     // accumulator columns kept in registers
-    const int tt = (warp - 8) >> 2;                // query tile of this warpgroup
-    const int quad = warp & 3;                     // TMEM lane quadrant
-    const int r = quad * 32 + lane;                // row within the tile
-    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    // Two threads per query row.  A softmax warp covers 16 rows of its TMEM lane
+    // quadrant; lane l < 16 takes the first half of every key block and of the
+    // accumulator columns of its row, lane l + 16 the second halves of the same
+    // row (.16x32bx2 TMEM accesses).
+    constexpr int kHK = BN / 2;          // keys of a block per thread
+    constexpr int kHD = D / 2;           // accumulator columns per thread
+    constexpr int kFr = kHD / 2;         // of which in registers (the rest in shared memory)
+    const int sw = warp - 8;             // softmax warp 0..15
+    const int tt = sw >> 3;              // query tile
+    const int sub = (sw >> 2) & 1;       // half of the lane quadrant
+    const int quad = warp & 3;           // TMEM lane quadrant
+    const int hh = lane >> 4;            // half of the keys / accumulator columns
+    const int r = quad * 32 + sub * 16 + (lane & 15);  // row within the tile
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32 + sub * 16) << 16;
     const uint32_t tA = tbase + tt * 256 + 128 + lane_off;
-    float4* Fs = reinterpret_cast<float4*>(smem + C::oF) + (tt * kRows + r) * (C::kFRow / 4);
+    float4* Fs = reinterpret_cast<float4*>(smem + C::oF) + ((tt * 2 + hh) * kRows + r) * (C::kFRow / 4);
     const float kLog2e = 1.4426950408889634f;
     // Arithmetic on pairs of fp32 (sm_100 f32x2 instructions: two lanes per
     // instruction, each rounded exactly like the scalar form).
@@ -398,10 +409,9 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const float2 k15x2 = make_float2(15.0f, 15.0f);
     uint32_t g = 0;
     bool ok = true;
-    float2 F2[kFh / 2];  // F[2i], F[2i+1]
+    float2 F2[kFr / 2];  // F[2i], F[2i+1] of this thread's columns
     // F += coef * (integer accumulator A); with reset, A is then set back to
-    // zero (its bits to 1.5 * 2^23).  The first half of the columns of F is in
-    // registers, the second half in shared memory.
+    // zero (its bits to 1.5 * 2^23).
     //
     // Without reset, A keeps accumulating across a change of the row maximum:
     // with segments s_k of P.V results between changes, A_k = s_1 + ... + s_k
@@ -411,37 +421,46 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     auto fold = [&](float coef, bool reset, int dump_t, bool dump_now) {
       const float2 w2 = make_float2(coef, coef);
 #pragma unroll
-      for (int c = 0; c < D; c += 32) {
+      for (int c = 0; c < kHD; c += 32) {
         uint32_t a[32];
-        tmem_ld32(tA + c, a);
-        if (c < kFh) {
+        tmem_ld_h<32, kHD>(tA + c, a);
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            F2[c / 2 + i] = __ffma2_rn(
-                w2, __fadd2_rn(make_float2(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1])), kNegMagic2),
-                F2[c / 2 + i]);
-        } else {
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const float4 f = Fs[(c - kFh) / 4 + q];
-            const float2 lo = __ffma2_rn(
-                w2, __fadd2_rn(make_float2(__uint_as_float(a[4 * q + 0]), __uint_as_float(a[4 * q + 1])), kNegMagic2),
-                make_float2(f.x, f.y));
-            const float2 hi = __ffma2_rn(
-                w2, __fadd2_rn(make_float2(__uint_as_float(a[4 * q + 2]), __uint_as_float(a[4 * q + 3])), kNegMagic2),
-                make_float2(f.z, f.w));
-            Fs[(c - kFh) / 4 + q] = make_float4(lo.x, lo.y, hi.x, hi.y);
+        for (int q = 0; q < 8; ++q) {
+          const int col = c + 4 * q;
+          const float2 lo = __fadd2_rn(make_float2(__uint_as_float(a[4 * q]), __uint_as_float(a[4 * q + 1])), kNegMagic2);
+          const float2 hi = __fadd2_rn(make_float2(__uint_as_float(a[4 * q + 2]), __uint_as_float(a[4 * q + 3])), kNegMagic2);
+          if (col < kFr) {
+            F2[col / 2] = __ffma2_rn(w2, lo, F2[col / 2]);
+            F2[col / 2 + 1] = __ffma2_rn(w2, hi, F2[col / 2 + 1]);
+          } else {
+            const float4 f = Fs[(col - kFr) / 4];
+            const float2 nl = __ffma2_rn(w2, lo, make_float2(f.x, f.y));
+            const float2 nh = __ffma2_rn(w2, hi, make_float2(f.z, f.w));
+            Fs[(col - kFr) / 4] = make_float4(nl.x, nl.y, nh.x, nh.y);
           }
         }
         if (DUMP && dump_now && prm.dump_acc) {
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            prm.dump_acc[(static_cast<size_t>(r) * nb + dump_t) * D + wide_to_dim(c + i)] =
+            prm.dump_acc[(static_cast<size_t>(r) * nb + dump_t) * D + wide_to_dim(hh * kHD + c + i)] =
                 (static_cast<int>(a[i]) - static_cast<int>(kMagic)) / 16;
         }
-        if (reset) tmem_fill32(tA + c, kMagic);
+        if (reset) {
+          uint32_t m[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) m[i] = kMagic;
+          tmem_st_h<32, kHD>(tA + c, m);
+        }
       }
     };
+    // The P.V accumulator starts at the bits of 1.5 * 2^23 (integer zero).
+    {
+      uint32_t m[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) m[i] = kMagic;
+#pragma unroll
+      for (int c = 0; c < kHD; c += 32) tmem_st_h<32, kHD>(tA + c, m);
+    }
     for (int item = blockIdx.x; item < prm.nitems && ok; item += gridDim.x) {
       const int bh = item / prm.npairs, pair = item % prm.npairs;
       const int qtile = pair * 2 + tt;
@@ -452,15 +471,12 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       const float2 cpi2 = make_float2(cpi, cpi);
       const bool dump_tile = DUMP && bh == prm.dump_bh && qtile == prm.dump_tile && row_ok;
 #pragma unroll
-      for (int i = 0; i < kFh / 2; ++i) F2[i] = make_float2(0.0f, 0.0f);
+      for (int i = 0; i < kFr / 2; ++i) F2[i] = make_float2(0.0f, 0.0f);
 #pragma unroll
-      for (int q = 0; q < kFh / 4; ++q) Fs[q] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      for (int q = 0; q < (kHD - kFr) / 4; ++q) Fs[q] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
       float m_run = -INFINITY, m_ref = 0.0f, w = 1.0f, Lf = 0.0f;
-      int Lrun = 0;   // code sum since the last fold (denominator)
-      int Labs = 0;   // code sum since the last reset of A (magnitude bound)
-      // fresh integer accumulator
-#pragma unroll
-      for (int c = 0; c < D; c += 32) tmem_fill32(tA + c, kMagic);
+      int Lrun = 0;   // code sum of the row since the last fold (denominator)
+      int Labs = 0;   // code sum of the row since the last reset of A (magnitude bound)
       for (int t = 0; t < nb; ++t, ++g) {
         const uint32_t buf = g & 1;
         const uint32_t tS = tbase + tt * 256 + buf * 64 + lane_off;
@@ -469,20 +485,21 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         tc_fence_after();
         const int ks = g % C::kKS;
         if (!(ok = wait_at(B.kw_full + ks, (g / C::kKS) & 1, abort_flag, 11u, g))) break;
-        const float4* ksc = reinterpret_cast<const float4*>(smem + C::oKsc) + ks * (BN / 4);
+        const float4* ksc = reinterpret_cast<const float4*>(smem + C::oKsc) + ks * (BN / 4) + hh * (kHK / 4);
         const int nvalid = min(BN, prm.N - t * BN);
-        // v = S_int * s_k for the whole block, in registers (256 S_int is exact
-        // in fp32 and s_k/256 a power-of-two scaling, so v is S_int * s_k
-        // rounded once).  Keys past N give NaN, which fmaxf skips.
-        uint32_t raw[BN];
-        tmem_ld<BN>(tS, raw);
-        if (dump_tile) {
-          for (int j = 0; j < nvalid; ++j)
-            if (prm.dump_s) prm.dump_s[static_cast<size_t>(r) * prm.N + t * BN + j] = static_cast<int32_t>(raw[j]) / 256;
+        // v = S_int * s_k for this thread's half of the block, in registers
+        // (256 S_int is exact in fp32 and s_k/256 a power-of-two scaling, so v
+        // is S_int * s_k rounded once).  Keys past N give NaN, which fmaxf skips.
+        uint32_t raw[kHK];
+        tmem_ld_h<kHK, kHK>(tS, raw);
+        if (dump_tile && prm.dump_s) {
+          for (int j = 0; j < kHK; ++j)
+            if (hh * kHK + j < nvalid)
+              prm.dump_s[static_cast<size_t>(r) * prm.N + t * BN + hh * kHK + j] = static_cast<int32_t>(raw[j]) / 256;
         }
-        float2 v2[BN / 2];
+        float2 v2[kHK / 2];
 #pragma unroll
-        for (int j = 0; j < BN; j += 4) {
+        for (int j = 0; j < kHK; j += 4) {
           const float4 sc = ksc[j / 4];
           v2[j / 2] = __fmul2_rn(make_float2(static_cast<float>(static_cast<int>(raw[j])),
                                              static_cast<float>(static_cast<int>(raw[j + 1]))),
@@ -491,7 +508,8 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                                                  static_cast<float>(static_cast<int>(raw[j + 3]))),
                                      make_float2(sc.z, sc.w));
         }
-        const float vmax = tree_max<BN>(reinterpret_cast<const float*>(v2));
+        float vmax = tree_max<kHK>(reinterpret_cast<const float*>(v2));
+        vmax = fmaxf(vmax, __shfl_xor_sync(0xFFFFFFFFu, vmax, 16));  // the row's other half
         const float m_blk = __fmul_rn(vmax, ci);
         const float m_new = fmaxf(m_run, m_blk);
         const bool grow = m_new > m_run;
@@ -499,9 +517,9 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const float2 nMp2 = make_float2(-Mp, -Mp);
         // P code c + 8 = rint(15 exp2(y)): adding 15 e to 1.5 * 2^23 rounds it
         // to an integer that lands in the low byte of the sum's bits.
-        uint32_t words[C::kKeysPV / 4];
+        uint32_t words[kHK / 4];
 #pragma unroll
-        for (int q = 0; q < BN / 4; ++q) {
+        for (int q = 0; q < kHK / 4; ++q) {
           const float2 x01 = __ffma2_rn(v2[2 * q], cpi2, nMp2);
           const float2 x23 = __ffma2_rn(v2[2 * q + 1], cpi2, nMp2);
           const float2 t01 = __ffma2_rn(k15x2, make_float2(ex2_approx(x01.x), ex2_approx(x01.y)), kMagic2);
@@ -511,8 +529,8 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         if (nvalid < BN) {  // last, ragged block: codes of keys past N are 0
 #pragma unroll
-          for (int q = 0; q < BN / 4; ++q) {
-            const int lim = nvalid - 4 * q;
+          for (int q = 0; q < kHK / 4; ++q) {
+            const int lim = nvalid - hh * kHK - 4 * q;
             words[q] &= lim >= 4 ? 0xFFFFFFFFu : (lim <= 0 ? 0u : (0xFFFFFFFFu >> (8 * (4 - lim))));
           }
         }
@@ -520,20 +538,25 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // word additions of up to 16 words cannot carry between bytes.
         uint32_t wsum = 0;
 #pragma unroll
-        for (int q = 0; q < BN / 4; ++q) wsum += words[q];
-        const int lq = static_cast<int>(__dp4a(wsum, 0x01010101u, 0u));  // unsigned bytes (up to 240)
+        for (int q = 0; q < kHK / 4; ++q) wsum += words[q];
+        int lq = static_cast<int>(__dp4a(wsum, 0x01010101u, 0u));  // unsigned bytes
+        lq += __shfl_xor_sync(0xFFFFFFFFu, lq, 16);
+        // P codes over the S columns they came from: word q of half hh is
+        // column hh * BN / 8 + q; P.V reads kKeysPV keys, those past BN are 0.
+        tmem_st_h<kHK / 4, kHK / 4>(tS, words);
+        if constexpr (C::kKeysPV > BN) {
+          constexpr int kZ = (C::kKeysPV - BN) / 8;
+          uint32_t zw[kZ];
 #pragma unroll
-        for (int q = BN / 4; q < C::kKeysPV / 4; ++q) words[q] = 0u;
-        if constexpr (C::kKeysPV / 4 == 16) tmem_st16(tS, words);
-        else if constexpr (C::kKeysPV / 4 == 8) tmem_st8(tS, words);
-        if (dump_tile && prm.dump_p) {
-          for (int j = 0; j < nvalid; ++j)
-            prm.dump_p[static_cast<size_t>(r) * prm.N + t * BN + j] =
-                static_cast<int8_t>(((words[j >> 2] >> (8 * (j & 3))) & 0xFF) - 8);
+          for (int q = 0; q < kZ; ++q) zw[q] = 0u;
+          tmem_st_h<kZ, kZ>(tS + BN / 4, zw);
         }
-        // Fold the integer accumulator into F when a row's maximum grows (its
-        // earlier codes used the old maximum) or its magnitude bound nears the
-        // exact range of the read-back (|acc| < 2^22).
+        if (dump_tile && prm.dump_p) {
+          for (int j = 0; j < kHK; ++j)
+            if (hh * kHK + j < nvalid)
+              prm.dump_p[static_cast<size_t>(r) * prm.N + t * BN + hh * kHK + j] =
+                  static_cast<int8_t>(((words[j >> 2] >> (8 * (j & 3))) & 0xFF) - 8);
+        }
         // Weight of the coming segment; a rescale moves the reference max.
         float w_new = w, sc = 1.0f;
         if (t == 0) {
@@ -561,9 +584,9 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           if (sc != 1.0f) {  // new reference maximum: rescale F and the denominator
             const float2 sc2 = make_float2(sc, sc);
 #pragma unroll
-            for (int i = 0; i < kFh / 2; ++i) F2[i] = __fmul2_rn(F2[i], sc2);
-            for (int q = 0; q < kFh / 4; ++q) {
-              float4 f = Fs[q];
+            for (int i = 0; i < kFr / 2; ++i) F2[i] = __fmul2_rn(F2[i], sc2);
+            for (int q = 0; q < (kHD - kFr) / 4; ++q) {
+              const float4 f = Fs[q];
               Fs[q] = make_float4(f.x * sc, f.y * sc, f.z * sc, f.w * sc);
             }
             Lf *= sc;
@@ -586,7 +609,7 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
       }
       if (!ok) break;
-      // Last block: fold the accumulator, normalise, store.
+      // Last block: fold the accumulator (and reset it), normalise, store.
       if (!(ok = wait_at(B.pv_done + tt * 2 + ((g - 1) & 1), ((g - 1) >> 1) & 1, abort_flag, 13u, g))) break;
       __syncwarp();
       tc_fence_after();
@@ -597,25 +620,30 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const float* sv = prm.sv + static_cast<size_t>(bh) * D;
         const float* Fsf = reinterpret_cast<const float*>(Fs);
         __nv_bfloat16* orow = prm.out + (static_cast<size_t>(bh) * prm.N + row) * D;
-        auto fget = [&](int i) -> float { return (i & 1) ? F2[i >> 1].y : F2[i >> 1].x; };
+        auto fget = [&](int i) -> float {  // column i of this thread's half
+          return i < kFr ? ((i & 1) ? F2[i >> 1].y : F2[i >> 1].x) : Fsf[i - kFr];
+        };
+        // Widened positions hh * D/2 + c + (4a + b) and + 16 hold channels
+        // d = hh * D/2 + c + 8a + 2b and d + 1.
 #pragma unroll
-        for (int c = 0; c < D; c += 32) {
+        for (int c = 0; c < kHD; c += 32) {
+          const int c0 = hh * kHD + c;
           uint32_t pk[16];
 #pragma unroll
           for (int a = 0; a < 4; ++a)
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
-              const int d = c + 8 * a + 2 * b;
-              const float f0 = c < kFh ? fget(c + 4 * a + b) : Fsf[c - kFh + 4 * a + b];
-              const float f1 = c < kFh ? fget(c + 16 + 4 * a + b) : Fsf[c - kFh + 16 + 4 * a + b];
-              const __nv_bfloat162 h = __floats2bfloat162_rn(f0 * __ldg(sv + d) * inv, f1 * __ldg(sv + d + 1) * inv);
-              pk[4 * a + b] = *reinterpret_cast<const uint32_t*>(&h);
+              const int d = c0 + 8 * a + 2 * b;
+              const float f0 = fget(c + 4 * a + b);
+              const float f1 = fget(c + 16 + 4 * a + b);
+              const __nv_bfloat162 h2 = __floats2bfloat162_rn(f0 * __ldg(sv + d) * inv, f1 * __ldg(sv + d + 1) * inv);
+              pk[4 * a + b] = *reinterpret_cast<const uint32_t*>(&h2);
             }
-          uint4* dst = reinterpret_cast<uint4*>(orow + c);
+          uint4* dst = reinterpret_cast<uint4*>(orow + c0);
 #pragma unroll
           for (int u = 0; u < 4; ++u) dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
         }
-        if (prm.lse) prm.lse[static_cast<size_t>(bh) * prm.N + row] = m_ref + logf(Lf * (1.0f / 15.0f));
+        if (prm.lse && hh == 0) prm.lse[static_cast<size_t>(bh) * prm.N + row] = m_ref + logf(Lf * (1.0f / 15.0f));
       }
     }
     if (!ok) set_status(kStatusTimeout);

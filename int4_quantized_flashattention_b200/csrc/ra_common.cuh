@@ -268,6 +268,77 @@ __device__ __forceinline__ void tmem_fill64_async(uint32_t taddr, uint32_t v) {
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// Half-warp shapes (.16x32bx2): lanes 0-15 of the warp access TMEM lanes
+// base..base+15 at columns c..c+N-1, lanes 16-31 the same TMEM lanes at
+// columns c+OFF..c+OFF+N-1 (base = the lane field of the address).  Waits are
+// fused as above.
+template <int N, int OFF> __device__ __forceinline__ void tmem_ld_h(uint32_t taddr, uint32_t* r);
+template <int N, int OFF> __device__ __forceinline__ void tmem_st_h(uint32_t taddr, const uint32_t* r);
+template <int OFF> __device__ __forceinline__ void tmem_ld_h2(uint32_t taddr, uint32_t* r) {
+  asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x2.b32 {%0,%1}, [%2], %3;\n\t"
+               "tcgen05.wait::ld.sync.aligned;"
+               : "=r"(r[0]), "=r"(r[1]) : "r"(taddr), "n"(OFF) : "memory");
+}
+template <int OFF> __device__ __forceinline__ void tmem_st_h2(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.16x32bx2.x2.b32 [%0], %1, {%2,%3};\n\t"
+               "tcgen05.wait::st.sync.aligned;"
+               :: "r"(taddr), "n"(OFF), "r"(r[0]), "r"(r[1]) : "memory");
+}
+template <int OFF> __device__ __forceinline__ void tmem_ld_h4(uint32_t taddr, uint32_t* r) {
+  asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x4.b32 {%0,%1,%2,%3}, [%4], %5;\n\t"
+               "tcgen05.wait::ld.sync.aligned;"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(taddr), "n"(OFF) : "memory");
+}
+template <int OFF> __device__ __forceinline__ void tmem_st_h4(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.16x32bx2.x4.b32 [%0], %1, {%2,%3,%4,%5};\n\t"
+               "tcgen05.wait::st.sync.aligned;"
+               :: "r"(taddr), "n"(OFF), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]) : "memory");
+}
+template <int OFF> __device__ __forceinline__ void tmem_ld_h8(uint32_t taddr, uint32_t* r) {
+  asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8], %9;\n\t"
+               "tcgen05.wait::ld.sync.aligned;"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]) : "r"(taddr), "n"(OFF) : "memory");
+}
+template <int OFF> __device__ __forceinline__ void tmem_st_h8(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.16x32bx2.x8.b32 [%0], %1, {%2,%3,%4,%5,%6,%7,%8,%9};\n\t"
+               "tcgen05.wait::st.sync.aligned;"
+               :: "r"(taddr), "n"(OFF), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]) : "memory");
+}
+template <int OFF> __device__ __forceinline__ void tmem_ld_h16(uint32_t taddr, uint32_t* r) {
+  asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16], %17;\n\t"
+               "tcgen05.wait::ld.sync.aligned;"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]) : "r"(taddr), "n"(OFF) : "memory");
+}
+template <int OFF> __device__ __forceinline__ void tmem_st_h16(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.16x32bx2.x16.b32 [%0], %1, {%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17};\n\t"
+               "tcgen05.wait::st.sync.aligned;"
+               :: "r"(taddr), "n"(OFF), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]) : "memory");
+}
+template <int OFF> __device__ __forceinline__ void tmem_ld_h32(uint32_t taddr, uint32_t* r) {
+  asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32], %33;\n\t"
+               "tcgen05.wait::ld.sync.aligned;"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]) : "r"(taddr), "n"(OFF) : "memory");
+}
+template <int OFF> __device__ __forceinline__ void tmem_st_h32(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.16x32bx2.x32.b32 [%0], %1, {%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33};\n\t"
+               "tcgen05.wait::st.sync.aligned;"
+               :: "r"(taddr), "n"(OFF), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]) : "memory");
+}
+template <int N, int OFF> __device__ __forceinline__ void tmem_ld_h(uint32_t taddr, uint32_t* r) {
+  if constexpr (N == 2) tmem_ld_h2<OFF>(taddr, r);
+  else if constexpr (N == 4) tmem_ld_h4<OFF>(taddr, r);
+  else if constexpr (N == 8) tmem_ld_h8<OFF>(taddr, r);
+  else if constexpr (N == 16) tmem_ld_h16<OFF>(taddr, r);
+  else tmem_ld_h32<OFF>(taddr, r);
+}
+template <int N, int OFF> __device__ __forceinline__ void tmem_st_h(uint32_t taddr, const uint32_t* r) {
+  if constexpr (N == 2) tmem_st_h2<OFF>(taddr, r);
+  else if constexpr (N == 4) tmem_st_h4<OFF>(taddr, r);
+  else if constexpr (N == 8) tmem_st_h8<OFF>(taddr, r);
+  else if constexpr (N == 16) tmem_st_h16<OFF>(taddr, r);
+  else tmem_st_h32<OFF>(taddr, r);
+}
+
 // ---------------------------------------------------------------- tcgen05.mma
 // D[tmem] (+)= A[smem desc] * B[smem desc]
 __device__ __forceinline__ void mma_i8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
@@ -301,6 +372,31 @@ __device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uin
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
       ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+
+// Warp-wide forms: every lane of the warp executes the call (so the operands
+// can live in uniform registers) and only lane 0 issues the instruction.
+__device__ __forceinline__ void mma_i8_ss_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, l;\n\t.reg .u32 ln;\n\tmov.u32 ln, %%laneid;\n\tsetp.eq.u32 l, ln, 0;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@l tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+__device__ __forceinline__ void mma_i8_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, l;\n\t.reg .u32 ln;\n\tmov.u32 ln, %%laneid;\n\tsetp.eq.u32 l, ln, 0;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@l tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+__device__ __forceinline__ void mma_commit_w(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred l;\n\t.reg .u32 ln;\n\tmov.u32 ln, %%laneid;\n\tsetp.eq.u32 l, ln, 0;\n\t"
+      "@l tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}"
+      ::"r"(smem_u32(bar)) : "memory");
 }
 
 // Arrives once on *bar when every tcgen05.mma issued so far by this thread has completed.
