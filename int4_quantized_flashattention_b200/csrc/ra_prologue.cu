@@ -108,6 +108,99 @@ __device__ __forceinline__ void rope_rotate8(const SegInfo& s, const float* tab_
   }
 }
 
+// Eight channels of one token as loaded from memory: one 16-byte word for bf16,
+// two for fp32.  Loads use the read-only path.
+template <bool kBf16>
+struct Raw8 {
+  uint4 u[kBf16 ? 1 : 2];
+};
+
+template <bool kBf16>
+__device__ __forceinline__ void load_raw8(const void* base, size_t elem_off, Raw8<kBf16>& r) {
+  if constexpr (kBf16) {
+    r.u[0] = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(base) + elem_off));
+  } else {
+    const uint4* p = reinterpret_cast<const uint4*>(static_cast<const float*>(base) + elem_off);
+    r.u[0] = __ldg(p);
+    r.u[1] = __ldg(p + 1);
+  }
+}
+
+template <bool kBf16>
+__device__ __forceinline__ void unpack8(const Raw8<kBf16>& r, float* x) {
+  if constexpr (kBf16) {
+    const uint32_t w[4] = {r.u[0].x, r.u[0].y, r.u[0].z, r.u[0].w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      x[2 * i] = __uint_as_float(w[i] << 16);
+      x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  } else {
+    x[0] = __uint_as_float(r.u[0].x); x[1] = __uint_as_float(r.u[0].y);
+    x[2] = __uint_as_float(r.u[0].z); x[3] = __uint_as_float(r.u[0].w);
+    x[4] = __uint_as_float(r.u[1].x); x[5] = __uint_as_float(r.u[1].y);
+    x[6] = __uint_as_float(r.u[1].z); x[7] = __uint_as_float(r.u[1].w);
+  }
+}
+
+// Table coefficients (a, b) of the 4 channel pairs [c0, c0 + 8) of a token at
+// grid position gp (one position per segment; out-of-grid positions are
+// reported and clamped so every table access stays in bounds).
+__device__ __forceinline__ void rope_coef8(const SegInfo& s, const float* tab_a, const float* tab_b, const int* gp,
+                                           int c0, float* ca, float* cb) {
+  int base[3];
+#pragma unroll
+  for (int j = 0; j < 3; ++j) {
+    int g = gp[j];
+    if (g < 0 || g >= s.grid[j]) {
+      atomicOr(&g_prologue_status, kStatusBadPosition);
+      g = g < 0 ? 0 : s.grid[j] - 1;
+    }
+    base[j] = s.toff[j] + g * (s.dj[j] >> 1);
+  }
+#pragma unroll
+  for (int pr = 0; pr < 4; ++pr) {
+    const int d = c0 + 2 * pr;
+    const int j = seg_of(s, d);
+    const int idx = (j == 0 ? base[0] : (j == 1 ? base[1] : base[2])) + ((d - s.off[j]) >> 1);
+    ca[pr] = __ldg(tab_a + idx);
+    cb[pr] = __ldg(tab_b + idx);
+  }
+}
+
+// The same arithmetic as rope_rotate8, from coefficients already loaded.
+__device__ __forceinline__ void rope_apply8(const SegInfo& s, int rot, const float* ca, const float* cb, int c0,
+                                            float* x, float* row) {
+#pragma unroll
+  for (int pr = 0; pr < 4; ++pr) {
+    const float a = ca[pr], b = cb[pr];
+    const float x0 = x[2 * pr], x1 = x[2 * pr + 1];
+    if (rot == 1) {
+      x[2 * pr] = __fadd_rn(__fmul_rn(x0, a), __fmul_rn(x1, b));
+      x[2 * pr + 1] = __fsub_rn(__fmul_rn(x0, b), __fmul_rn(x1, a));
+    } else {
+      x[2 * pr] = __fsub_rn(__fmul_rn(x0, a), __fmul_rn(x1, b));
+      x[2 * pr + 1] = __fadd_rn(__fmul_rn(x0, b), __fmul_rn(x1, a));
+    }
+  }
+  if (rot == 2) {
+    const float r2 = 0.70710678118654752440f;  // fp32 rounding of 1/sqrt(2)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) row[c0 + i] = x[i];
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int d = c0 + i;
+      const int j = seg_of(s, d);
+      const int h = s.dj[j] >> 1;
+      const int t = (d - s.off[j]) >> 1;
+      const float u = row[s.off[j] + t], w = row[s.off[j] + t + h];
+      x[i] = (d - s.off[j]) & 1 ? __fmul_rn(__fsub_rn(u, w), r2) : __fmul_rn(__fadd_rn(u, w), r2);
+    }
+    __syncwarp();
+  }
+}
+
 // rint(y) for |y| < 2^22 with ties to even: adding 1.5 * 2^23 rounds to an integer.
 __device__ __forceinline__ int rint_small(float y) {
   return __float_as_int(__fadd_rn(y, 12582912.0f)) - 0x4B400000;
@@ -166,7 +259,9 @@ __global__ void rope_table_kernel(SegInfo s, int total, double theta, int rot, f
 }
 
 // Pass 1: per chunk of tokens, fp64 channel sums of the rotated K and channel
-// maxima of |V|.
+// maxima of |V|.  Each thread loads the next token's K, V and position before
+// working on the current one.
+template <bool kBf16>
 __global__ void __launch_bounds__(kThreads) prologue_reduce_kernel(PrologueArgs a) {
   __shared__ float rows[kThreads / 32][4][128];
   __shared__ double red_s[kThreads][8];
@@ -175,26 +270,43 @@ __global__ void __launch_bounds__(kThreads) prologue_reduce_kernel(PrologueArgs 
   const int lpt = a.D >> 3, tpw = 32 / lpt;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tok_in_warp = lane / lpt, c0 = (lane % lpt) * 8;
+  const int step = (kThreads / 32) * tpw, iters = kChunk / step;
   double ks[8];
   float vm[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) { ks[i] = 0.0; vm[i] = 0.0f; }
-  const int n0 = chunk * kChunk;
   const size_t head = static_cast<size_t>(bh) * a.N * a.D;
-  for (int base = n0; base < n0 + kChunk; base += (kThreads / 32) * tpw) {
-    const int n = base + warp * tpw + tok_in_warp;
+  int n = chunk * kChunk + warp * tpw + tok_in_warp;
+  Raw8<kBf16> rk{}, rv{};
+  int gp[3] = {0, 0, 0};
+  auto fetch = [&](int nn) {
+    if (nn < a.N) {
+      load_raw8<kBf16>(a.k, head + static_cast<size_t>(nn) * a.D + c0, rk);
+      load_raw8<kBf16>(a.v, head + static_cast<size_t>(nn) * a.D + c0, rv);
+#pragma unroll
+      for (int j = 0; j < 3; ++j) gp[j] = __ldg(a.pos + 3 * nn + j);
+    }
+  };
+  fetch(n);
+  for (int it = 0; it < iters; ++it) {
     const bool ok = n < a.N;
-    float x[8], y[8];
+    const Raw8<kBf16> ck = rk, cv = rv;
+    const int g3[3] = {gp[0], gp[1], gp[2]};
+    n += step;
+    if (it + 1 < iters) fetch(n);
+    float x[8], y[8], ca[4], cb[4];
     if (ok) {
-      load8(a.k, head + static_cast<size_t>(n) * a.D + c0, a.dtype, x);
-      load8(a.v, head + static_cast<size_t>(n) * a.D + c0, a.dtype, y);
+      unpack8<kBf16>(ck, x);
+      unpack8<kBf16>(cv, y);
     } else {
 #pragma unroll
       for (int i = 0; i < 8; ++i) { x[i] = 0.0f; y[i] = 0.0f; }
     }
-    // rope_rotate8 synchronises the warp for the half rotation, so every lane
-    // takes part; lanes past N carry zeros and position 0.
-    rope_rotate8(a.s, a.tab_a, a.tab_b, a.pos, ok ? n : 0, a.rot, c0, x, rows[warp][tok_in_warp]);
+    // Every lane takes part (the half rotation synchronises the warp); lanes
+    // past N carry zeros and the position of token 0's default.
+    const int z3[3] = {0, 0, 0};
+    rope_coef8(a.s, a.tab_a, a.tab_b, ok ? g3 : z3, c0, ca, cb);
+    rope_apply8(a.s, a.rot, ca, cb, c0, x, rows[warp][tok_in_warp]);
     if (ok) {
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -239,7 +351,12 @@ __global__ void prologue_finalize_kernel(PrologueArgs a) {
 }
 
 // Pass 2: quantise.  Q, K: rotate (K also smoothed), per-token scale and codes.
-// V: per-channel codes, column sums per key block.
+// V: per-channel codes, column sums per key block.  Each thread loads the next
+// token's Q, K, V and position before working on the current one; Q and K share
+// the RoPE coefficients of the token.  Column sums are kept per thread while a
+// warp stays in one key block, then combined across the warp's tokens and
+// added to shared memory.
+template <bool kBf16>
 __global__ void __launch_bounds__(kThreads) prologue_quant_kernel(PrologueArgs a) {
   __shared__ float rows[kThreads / 32][4][128];
   __shared__ int csum[kChunk / 16][128];
@@ -247,6 +364,7 @@ __global__ void __launch_bounds__(kThreads) prologue_quant_kernel(PrologueArgs a
   const int lpt = a.D >> 3, tpw = 32 / lpt;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tok_in_warp = lane / lpt, c0 = (lane % lpt) * 8;
+  const int step = (kThreads / 32) * tpw, iters = kChunk / step;
   const int nblk = kChunk / a.block_k;
   for (int i = threadIdx.x; i < nblk * a.D; i += kThreads) csum[i / a.D][i % a.D] = 0;
   float kmean[8], vinv[8];
@@ -259,21 +377,61 @@ __global__ void __launch_bounds__(kThreads) prologue_quant_kernel(PrologueArgs a
   const int n0 = chunk * kChunk;
   const size_t head = static_cast<size_t>(bh) * a.N * a.D;
   const size_t head4 = static_cast<size_t>(bh) * a.N * (a.D / 2);
-  for (int base = n0; base < n0 + kChunk; base += (kThreads / 32) * tpw) {
-    const int n = base + warp * tpw + tok_in_warp;
+  int n = n0 + warp * tpw + tok_in_warp;
+  Raw8<kBf16> rq{}, rk{}, rv{};
+  int gp[3] = {0, 0, 0};
+  auto fetch = [&](int nn) {
+    if (nn < a.N) {
+      const size_t o = head + static_cast<size_t>(nn) * a.D + c0;
+      load_raw8<kBf16>(a.q, o, rq);
+      load_raw8<kBf16>(a.k, o, rk);
+      load_raw8<kBf16>(a.v, o, rv);
+#pragma unroll
+      for (int j = 0; j < 3; ++j) gp[j] = __ldg(a.pos + 3 * nn + j);
+    }
+  };
+  fetch(n);
+  int cacc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  int cblk = (warp * tpw) / a.block_k;  // key block of this warp's tokens in iteration 0
+  // Adds this warp's per-thread column sums of block cblk to shared memory:
+  // lanes holding the same channels (lpt apart) are combined first.
+  auto flush = [&]() {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      for (int o = lpt; o < 32; o <<= 1) cacc[i] += __shfl_xor_sync(0xFFFFFFFFu, cacc[i], o);
+    if (tok_in_warp == 0) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (cacc[i] != 0) atomicAdd(&csum[cblk][c0 + i], cacc[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) cacc[i] = 0;
+  };
+  for (int it = 0; it < iters; ++it) {
     const bool ok = n < a.N;
-    const int nn = ok ? n : 0;
-    float xq[8], xk[8], xv[8];
+    const int ncur = n;
+    const Raw8<kBf16> cq = rq, ck = rk, cv = rv;
+    const int g3[3] = {gp[0], gp[1], gp[2]};
+    n += step;
+    if (it + 1 < iters) fetch(n);
+    const int blk = (it * step + warp * tpw) / a.block_k;  // the same for the warp's tokens
+    if (blk != cblk) {
+      flush();
+      cblk = blk;
+    }
+    float xq[8], xk[8], xv[8], ca[4], cb[4];
     if (ok) {
-      load8(a.q, head + static_cast<size_t>(n) * a.D + c0, a.dtype, xq);
-      load8(a.k, head + static_cast<size_t>(n) * a.D + c0, a.dtype, xk);
-      load8(a.v, head + static_cast<size_t>(n) * a.D + c0, a.dtype, xv);
+      unpack8<kBf16>(cq, xq);
+      unpack8<kBf16>(ck, xk);
+      unpack8<kBf16>(cv, xv);
     } else {
 #pragma unroll
       for (int i = 0; i < 8; ++i) { xq[i] = 0.0f; xk[i] = 0.0f; xv[i] = 0.0f; }
     }
-    rope_rotate8(a.s, a.tab_a, a.tab_b, a.pos, nn, a.rot, c0, xq, rows[warp][tok_in_warp]);
-    rope_rotate8(a.s, a.tab_a, a.tab_b, a.pos, nn, a.rot, c0, xk, rows[warp][tok_in_warp]);
+    const int z3[3] = {0, 0, 0};
+    rope_coef8(a.s, a.tab_a, a.tab_b, ok ? g3 : z3, c0, ca, cb);
+    rope_apply8(a.s, a.rot, ca, cb, c0, xq, rows[warp][tok_in_warp]);
+    rope_apply8(a.s, a.rot, ca, cb, c0, xk, rows[warp][tok_in_warp]);
     float mq = 0.0f, mk = 0.0f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -283,30 +441,29 @@ __global__ void __launch_bounds__(kThreads) prologue_quant_kernel(PrologueArgs a
     }
     mq = group_max(mq, lpt);
     mk = group_max(mk, lpt);
-    int cq[8], ck[8], cv[8];
+    int cq8[8], ck8[8], cv8[8];
     const float iq = mq == 0.0f ? 0.0f : __fdiv_rn(7.0f, mq);
     const float ik = mk == 0.0f ? 0.0f : __fdiv_rn(7.0f, mk);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      cq[i] = quant4(xq[i], iq);
-      ck[i] = quant4(xk[i], ik);
-      cv[i] = quant4(xv[i], vinv[i]);
+      cq8[i] = quant4(xq[i], iq);
+      ck8[i] = quant4(xk[i], ik);
+      cv8[i] = quant4(xv[i], vinv[i]);
     }
     if (ok) {
-      const size_t o4 = head4 + static_cast<size_t>(n) * (a.D / 2) + (c0 >> 1);
-      *reinterpret_cast<uint32_t*>(a.q4 + o4) = pack8(cq);
-      *reinterpret_cast<uint32_t*>(a.k4 + o4) = pack8(ck);
-      *reinterpret_cast<uint32_t*>(a.v4 + o4) = pack8(cv);
+      const size_t o4 = head4 + static_cast<size_t>(ncur) * (a.D / 2) + (c0 >> 1);
+      *reinterpret_cast<uint32_t*>(a.q4 + o4) = pack8(cq8);
+      *reinterpret_cast<uint32_t*>(a.k4 + o4) = pack8(ck8);
+      *reinterpret_cast<uint32_t*>(a.v4 + o4) = pack8(cv8);
       if (c0 == 0) {
-        a.sq[static_cast<size_t>(bh) * a.N + n] = __fdiv_rn(mq, 7.0f);
-        a.sk[static_cast<size_t>(bh) * a.N + n] = __fdiv_rn(mk, 7.0f);
+        a.sq[static_cast<size_t>(bh) * a.N + ncur] = __fdiv_rn(mq, 7.0f);
+        a.sk[static_cast<size_t>(bh) * a.N + ncur] = __fdiv_rn(mk, 7.0f);
       }
-      const int blk = (n - n0) / a.block_k;
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        if (cv[i] != 0) atomicAdd(&csum[blk][c0 + i], cv[i]);
+      for (int i = 0; i < 8; ++i) cacc[i] += cv8[i];
     }
   }
+  flush();
   __syncthreads();
   const int nb_total = (a.N + a.block_k - 1) / a.block_k;
   for (int i = threadIdx.x; i < nblk * a.D; i += kThreads) {
@@ -413,11 +570,13 @@ cudaError_t launch_prologue(const ra_problem& p, int dtype, const void* q, const
   cudaError_t e = launch_tables(p, p.rot, const_cast<float*>(a.tab_a), const_cast<float*>(a.tab_b), st);
   if (e != cudaSuccess) return e;
   const dim3 grid(a.nchunk, p.B * p.H);
-  prologue_reduce_kernel<<<grid, kThreads, 0, st>>>(a);
+  if (dtype == 1) prologue_reduce_kernel<true><<<grid, kThreads, 0, st>>>(a);
+  else prologue_reduce_kernel<false><<<grid, kThreads, 0, st>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   prologue_finalize_kernel<<<p.B * p.H, 128, 0, st>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  prologue_quant_kernel<<<grid, kThreads, 0, st>>>(a);
+  if (dtype == 1) prologue_quant_kernel<true><<<grid, kThreads, 0, st>>>(a);
+  else prologue_quant_kernel<false><<<grid, kThreads, 0, st>>>(a);
   return cudaGetLastError();
 }
 
