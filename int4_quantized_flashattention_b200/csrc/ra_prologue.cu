@@ -262,7 +262,7 @@ __global__ void rope_table_kernel(SegInfo s, int total, double theta, int rot, f
 // maxima of |V|.  Each thread loads the next token's K, V and position before
 // working on the current one.
 template <bool kBf16>
-__global__ void __launch_bounds__(kThreads) prologue_reduce_kernel(PrologueArgs a) {
+__global__ void __launch_bounds__(kThreads, 3) prologue_reduce_kernel(PrologueArgs a) {
   __shared__ float rows[kThreads / 32][4][128];
   __shared__ double red_s[kThreads][8];
   __shared__ float red_m[kThreads][8];
@@ -357,7 +357,7 @@ __global__ void prologue_finalize_kernel(PrologueArgs a) {
 // warp stays in one key block, then combined across the warp's tokens and
 // added to shared memory.
 template <bool kBf16>
-__global__ void __launch_bounds__(kThreads) prologue_quant_kernel(PrologueArgs a) {
+__global__ void __launch_bounds__(kThreads, 3) prologue_quant_kernel(PrologueArgs a) {
   __shared__ float rows[kThreads / 32][4][128];
   __shared__ int csum[kChunk / 16][128];
   const int bh = blockIdx.y, chunk = blockIdx.x;
