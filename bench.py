@@ -231,6 +231,27 @@ def run_ours(args, rank, world, local_rank):
     h2d = sum(host[n].numel() * 2 for n in ("q", "k", "v")) + pos_h.numel() * 4
     d2h = out_h.numel() * 2
 
+    # The bf16 fallback (plain RoPE'd q, k and v in bf16), timed on its own:
+    # not part of the INT4 step, reported against the bf16 tensor peak.
+    qr, kr = ra.rope_bf16(p, q, k, pos, workspace=ws)
+    out_b = torch.empty_like(out)
+    for _ in range(2):
+        ra.attn_bf16_fallback(p, qr, kr, v, out=out_b)
+    torch.cuda.synchronize(dev)
+    fb = []
+    for _ in range(max(3, args.steps // 4)):
+        a0 = torch.cuda.Event(enable_timing=True)
+        a1 = torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        ra.attn_bf16_fallback(p, qr, kr, v, out=out_b)
+        a1.record(stream)
+        torch.cuda.synchronize(dev)
+        fb.append(a0.elapsed_time(a1))
+    if ra.sync_status() != 0:
+        raise RuntimeError("device status not ok after the bf16 fallback")
+    fb_ms = statistics.median(fb)
+    del qr, kr, out_b
+
     ops = wl.attn_ops()
     ms_step = total_ms / args.steps
     value = world * ops / (ms_step * 1e-3) / 1e12
@@ -256,6 +277,9 @@ def run_ours(args, rank, world, local_rank):
                      "peak_gbs": pk["hbm_gbs"], "frac": round(pro_bytes / (pro_med * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
                      "ratio_to_attention": round(pro_med / att_med, 4)},
         "attention_ms": round(att_med, 4),
+        "bf16_fallback": {"ms": round(fb_ms, 4), "tflops": round(ops / (fb_ms * 1e-3) / 1e12, 1),
+                          "peak": pk["bf16_tflops"], "frac": round(ops / (fb_ms * 1e-3) / 1e12 / pk["bf16_tflops"], 4),
+                          "kernel": "attn_bf16_kernel", "note": "4N^2DH flops of bf16 attention on the RoPE'd inputs"},
         "gpu_launches": KERNELS_PER_STEP * args.steps,
         "clocks": clk.summary(),
     }
