@@ -138,6 +138,27 @@ def cpu_baseline(wl, target_s: float = 15.0, x=None):
                       f"attention of {rows} query rows over all {wl.N} keys; {t:.1f} s of CPU time"}
 
 
+def _attn_traffic():
+    """DRAM bytes per attention launch from the committed ncu summary, or None
+    when the attention kernel's sources changed since those counters were taken."""
+    import hashlib
+    import re
+    path = os.path.join(ROOT, "profiles", "launches_wan.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    mt = re.search(r"traffic_bytes_per_launch: (\d+)", text)
+    mh = re.search(r"kernel_sources_sha256: ([0-9a-f]{64})", text)
+    if not mt or not mh:
+        return None
+    h = hashlib.sha256()
+    for f in ("ra_attn_int4.cu", "ra_common.cuh"):
+        with open(os.path.join(ROOT, "int4_quantized_flashattention_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return int(mt.group(1)) if h.hexdigest() == mh.group(1) else None
+
+
 def run_ours(args, rank, world, local_rank):
     import numpy as np
     import torch
@@ -271,7 +292,7 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {"bound": "tensor", "kernel": "attn_int4_kernel", "achieved": round(achieved, 1),
                      "peak": round(int8_peak, 1), "unit": "TFLOP/s", "frac": round(achieved / int8_peak, 4),
                      "peak_source": f"2 x {pk['source']} bf16 burst {pk['bf16_tflops']} TFLOP/s (int8 ops/s)",
-                     "traffic": None},
+                     "traffic": _attn_traffic() if args.workload == "wan" else None},
         "prologue": {"ms": round(pro_med, 4), "bytes": pro_bytes,
                      "achieved_gbs": round(pro_bytes / (pro_med * 1e-3) / 1e9, 1),
                      "peak_gbs": pk["hbm_gbs"], "frac": round(pro_bytes / (pro_med * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
