@@ -339,6 +339,14 @@ template <int N, int OFF> __device__ __forceinline__ void tmem_st_h(uint32_t tad
   else tmem_st_h32<OFF>(taddr, r);
 }
 
+// Bulk asynchronous copy global -> shared (no multicast), completing `bytes`
+// of transaction count on the mbarrier.  Addresses 16-byte aligned, size a
+// multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
+}
+
 // ---------------------------------------------------------------- tcgen05.mma
 // D[tmem] (+)= A[smem desc] * B[smem desc]
 __device__ __forceinline__ void mma_i8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,

@@ -143,26 +143,40 @@ __device__ __forceinline__ void unpack8(const Raw8<kBf16>& r, float* x) {
   }
 }
 
-// Table coefficients (a, b) of the 4 channel pairs [c0, c0 + 8) of a token at
-// grid position gp (one position per segment; out-of-grid positions are
-// reported and clamped so every table access stays in bounds).
-__device__ __forceinline__ void rope_coef8(const SegInfo& s, const float* tab_a, const float* tab_b, const int* gp,
-                                           int c0, float* ca, float* cb) {
-  int base[3];
+// Per-thread constants of the RoPE table lookup: the segment and the pair of
+// each of the thread's 4 channel pairs, computed once.
+struct RopePlan {
+  int seg[4], off[4], stride[4];
+  __device__ __forceinline__ void init(const SegInfo& s, int c0) {
+#pragma unroll
+    for (int pr = 0; pr < 4; ++pr) {
+      const int d = c0 + 2 * pr;
+      const int j = seg_of(s, d);
+      seg[pr] = j;
+      off[pr] = s.toff[j] + ((d - s.off[j]) >> 1);
+      stride[pr] = s.dj[j] >> 1;
+    }
+  }
+};
+
+// Table coefficients (a, b) of the thread's 4 channel pairs for a token at grid
+// position gp (one position per segment; out-of-grid positions are reported
+// and clamped so every table access stays in bounds).
+__device__ __forceinline__ void rope_coef8p(const SegInfo& s, const RopePlan& rp, const float* tab_a,
+                                            const float* tab_b, const int* gp, float* ca, float* cb) {
+  int g[3];
 #pragma unroll
   for (int j = 0; j < 3; ++j) {
-    int g = gp[j];
-    if (g < 0 || g >= s.grid[j]) {
+    g[j] = gp[j];
+    if (g[j] < 0 || g[j] >= s.grid[j]) {
       atomicOr(&g_prologue_status, kStatusBadPosition);
-      g = g < 0 ? 0 : s.grid[j] - 1;
+      g[j] = g[j] < 0 ? 0 : s.grid[j] - 1;
     }
-    base[j] = s.toff[j] + g * (s.dj[j] >> 1);
   }
 #pragma unroll
   for (int pr = 0; pr < 4; ++pr) {
-    const int d = c0 + 2 * pr;
-    const int j = seg_of(s, d);
-    const int idx = (j == 0 ? base[0] : (j == 1 ? base[1] : base[2])) + ((d - s.off[j]) >> 1);
+    const int gj = rp.seg[pr] == 0 ? g[0] : (rp.seg[pr] == 1 ? g[1] : g[2]);
+    const int idx = rp.off[pr] + gj * rp.stride[pr];
     ca[pr] = __ldg(tab_a + idx);
     cb[pr] = __ldg(tab_b + idx);
   }
@@ -201,21 +215,21 @@ __device__ __forceinline__ void rope_apply8(const SegInfo& s, int rot, const flo
   }
 }
 
-// rint(y) for |y| < 2^22 with ties to even: adding 1.5 * 2^23 rounds to an integer.
-__device__ __forceinline__ int rint_small(float y) {
-  return __float_as_int(__fadd_rn(y, 12582912.0f)) - 0x4B400000;
+
+// Bits of 1.5 * 2^23 + clamp(rint(x * inv), -7, 7): clamping before rounding
+// gives the same integer (rint is monotone and +-7 are integers); the code is
+// the value minus 0x4B400000, and its low 4 bits are the two's complement nibble.
+__device__ __forceinline__ uint32_t quant4_bits(float x, float inv) {
+  const float y = fminf(fmaxf(__fmul_rn(x, inv), -7.0f), 7.0f);
+  return __float_as_uint(__fadd_rn(y, 12582912.0f));
 }
 
-__device__ __forceinline__ int quant4(float x, float inv) {
-  int c = rint_small(__fmul_rn(x, inv));
-  return c > 7 ? 7 : (c < -7 ? -7 : c);
-}
-
-__device__ __forceinline__ uint32_t pack8(const int* c) {
-  uint32_t w = 0;
+// Packs the nibbles of eight quant4_bits results, element 2t in the low nibble.
+__device__ __forceinline__ uint32_t pack8_bits(const uint32_t* b) {
+  uint32_t p[4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) w |= static_cast<uint32_t>(c[i] & 0xF) << (4 * i);
-  return w;
+  for (int j = 0; j < 4; ++j) p[j] = (b[2 * j] & 0x0Fu) | ((b[2 * j + 1] << 4) & ~0x0Fu);  // byte 0 is the pair
+  return __byte_perm(__byte_perm(p[0], p[1], 0x0040), __byte_perm(p[2], p[3], 0x0040), 0x5410);
 }
 
 // Max over the D/8 threads of a token (a contiguous lane group of size lpt).
@@ -258,74 +272,133 @@ __global__ void rope_table_kernel(SegInfo s, int total, double theta, int rot, f
   }
 }
 
+// Rows of kSub tokens of the input tensors are staged in shared memory by bulk
+// asynchronous copies, kStg sub-chunks ahead of the threads that use them, so
+// each SM keeps tens of kilobytes of loads in flight.  Thread 0 issues the
+// copies; every stage has one mbarrier that completes on the copied bytes.
+constexpr int kSub = 32;   // tokens per stage
+constexpr int kStg = 2;    // stages
+
+template <bool kBf16, int NT>
+struct StageIO {
+  static constexpr int kEl = kBf16 ? 2 : 4;
+  // Issues the copies of sub-chunk sc (tokens n0 + sc*kSub ...) of NT tensors
+  // into stage sc % kStg; a sub-chunk past N only completes the barrier.
+  static __device__ __forceinline__ void issue(const void* const* src, size_t head, int D, int N, int n0, int sc,
+                                               uint8_t* stg, uint64_t* full) {
+    const int s = sc % kStg;
+    const int t0 = n0 + sc * kSub;
+    const int cnt = min(kSub, N - t0);
+    if (cnt <= 0) {
+      mbar_arrive(full + s);
+      return;
+    }
+    const uint32_t tb = kSub * D * kEl, bytes = static_cast<uint32_t>(cnt) * D * kEl;
+    mbar_arrive_expect_tx(full + s, NT * bytes);
+    for (int i = 0; i < NT; ++i)
+      bulk_g2s(stg + (s * NT + i) * tb, static_cast<const uint8_t*>(src[i]) + (head + static_cast<size_t>(t0) * D) * kEl,
+               bytes, full + s);
+  }
+  // This thread's 8 channels of token ti of tensor i in stage s.
+  static __device__ __forceinline__ void read(const uint8_t* stg, int D, int s, int i, int ti, int c0, Raw8<kBf16>& r) {
+    const uint8_t* p = stg + ((s * NT + i) * kSub + ti) * D * kEl + c0 * kEl;
+    r.u[0] = *reinterpret_cast<const uint4*>(p);
+    if constexpr (!kBf16) r.u[1] = *reinterpret_cast<const uint4*>(p + 16);
+  }
+  static constexpr int stage_bytes(int D) { return NT * kSub * D * kEl; }
+};
+
+// Waits (bounded) for stage s's copies; returns false in every thread of the
+// CTA if any thread gave up.
+__device__ __forceinline__ bool stage_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  const int r = mbar_wait_ex(bar, parity, abort, 64u);
+  return !__syncthreads_or(r <= 0);
+}
+
 // Pass 1: per chunk of tokens, fp64 channel sums of the rotated K and channel
-// maxima of |V|.  Each thread loads the next token's K, V and position before
-// working on the current one.
+// maxima of |V|.
 template <bool kBf16>
 __global__ void __launch_bounds__(kThreads, 3) prologue_reduce_kernel(PrologueArgs a) {
+  using IO = StageIO<kBf16, 2>;
   __shared__ float rows[kThreads / 32][4][128];
-  __shared__ double red_s[kThreads][8];
-  __shared__ float red_m[kThreads][8];
+  __shared__ uint64_t full[kStg];
+  __shared__ int abort_flag;
+  extern __shared__ __align__(128) uint8_t stg[];
   const int bh = blockIdx.y, chunk = blockIdx.x;
   const int lpt = a.D >> 3, tpw = 32 / lpt;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tok_in_warp = lane / lpt, c0 = (lane % lpt) * 8;
-  const int step = (kThreads / 32) * tpw, iters = kChunk / step;
+  const int step = (kThreads / 32) * tpw;
+  const int n0 = chunk * kChunk;
+  const size_t head = static_cast<size_t>(bh) * a.N * a.D;
+  const void* src[2] = {a.k, a.v};
+  RopePlan rp;
+  rp.init(a.s, c0);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStg; ++s) mbar_init(full + s, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0)
+    for (int sc = 0; sc < kStg; ++sc) IO::issue(src, head, a.D, a.N, n0, sc, stg, full);
   double ks[8];
   float vm[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) { ks[i] = 0.0; vm[i] = 0.0f; }
-  const size_t head = static_cast<size_t>(bh) * a.N * a.D;
-  int n = chunk * kChunk + warp * tpw + tok_in_warp;
-  Raw8<kBf16> rk{}, rv{};
-  int gp[3] = {0, 0, 0};
-  auto fetch = [&](int nn) {
-    if (nn < a.N) {
-      load_raw8<kBf16>(a.k, head + static_cast<size_t>(nn) * a.D + c0, rk);
-      load_raw8<kBf16>(a.v, head + static_cast<size_t>(nn) * a.D + c0, rv);
+  bool ok = true;
+  for (int sc = 0; sc < kChunk / kSub && ok; ++sc) {
+    const int s = sc % kStg;
+    if (!(ok = stage_wait(full + s, (sc / kStg) & 1, &abort_flag))) break;
+    for (int ti = warp * tpw + tok_in_warp; ti - tok_in_warp < kSub; ti += step) {
+      const int n = n0 + sc * kSub + ti;
+      const bool valid = n < a.N;
+      float x[8], y[8], ca[4], cb[4];
+      int gp[3] = {0, 0, 0};
+      if (valid) {
+        Raw8<kBf16> rk, rv;
+        IO::read(stg, a.D, s, 0, ti, c0, rk);
+        IO::read(stg, a.D, s, 1, ti, c0, rv);
+        unpack8<kBf16>(rk, x);
+        unpack8<kBf16>(rv, y);
 #pragma unroll
-      for (int j = 0; j < 3; ++j) gp[j] = __ldg(a.pos + 3 * nn + j);
-    }
-  };
-  fetch(n);
-  for (int it = 0; it < iters; ++it) {
-    const bool ok = n < a.N;
-    const Raw8<kBf16> ck = rk, cv = rv;
-    const int g3[3] = {gp[0], gp[1], gp[2]};
-    n += step;
-    if (it + 1 < iters) fetch(n);
-    float x[8], y[8], ca[4], cb[4];
-    if (ok) {
-      unpack8<kBf16>(ck, x);
-      unpack8<kBf16>(cv, y);
-    } else {
+        for (int j = 0; j < 3; ++j) gp[j] = __ldg(a.pos + 3 * n + j);
+      } else {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) { x[i] = 0.0f; y[i] = 0.0f; }
-    }
-    // Every lane takes part (the half rotation synchronises the warp); lanes
-    // past N carry zeros and the position of token 0's default.
-    const int z3[3] = {0, 0, 0};
-    rope_coef8(a.s, a.tab_a, a.tab_b, ok ? g3 : z3, c0, ca, cb);
-    rope_apply8(a.s, a.rot, ca, cb, c0, x, rows[warp][tok_in_warp]);
-    if (ok) {
+        for (int i = 0; i < 8; ++i) { x[i] = 0.0f; y[i] = 0.0f; }
+      }
+      // Every lane takes part (the half rotation synchronises the warp).
+      rope_coef8p(a.s, rp, a.tab_a, a.tab_b, gp, ca, cb);
+      rope_apply8(a.s, a.rot, ca, cb, c0, x, rows[warp][tok_in_warp]);
+      if (valid) {
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        ks[i] += static_cast<double>(x[i]);
-        vm[i] = fmaxf(vm[i], fabsf(y[i]));
+        for (int i = 0; i < 8; ++i) {
+          ks[i] += static_cast<double>(x[i]);
+          vm[i] = fmaxf(vm[i], fabsf(y[i]));
+        }
       }
     }
+    __syncthreads();  // stage s consumed
+    if (threadIdx.x == 0 && sc + kStg < kChunk / kSub) IO::issue(src, head, a.D, a.N, n0, sc + kStg, stg, full);
   }
+  if (!ok) {
+    if (threadIdx.x == 0) atomicOr(&g_prologue_status, kStatusTimeout);
+    return;
+  }
+  // Per-thread partials to shared memory (reusing the stage buffers), folded
+  // in thread order per channel.
+  double* red_s = reinterpret_cast<double*>(stg);
+  float* red_m = reinterpret_cast<float*>(stg + kThreads * 8 * sizeof(double));
 #pragma unroll
-  for (int i = 0; i < 8; ++i) { red_s[threadIdx.x][i] = ks[i]; red_m[threadIdx.x][i] = vm[i]; }
+  for (int i = 0; i < 8; ++i) { red_s[threadIdx.x * 8 + i] = ks[i]; red_m[threadIdx.x * 8 + i] = vm[i]; }
   __syncthreads();
-  // Threads t with t % lpt == c hold channels [8c, 8c+8); fold them in thread order.
   for (int d = threadIdx.x; d < a.D; d += kThreads) {
     const int c = d >> 3, i = d & 7;
     double sum = 0.0;
     float mx = 0.0f;
     for (int t = c; t < kThreads; t += lpt) {
-      sum += red_s[t][i];
-      mx = fmaxf(mx, red_m[t][i]);
+      sum += red_s[t * 8 + i];
+      mx = fmaxf(mx, red_m[t * 8 + i]);
     }
     const size_t o = (static_cast<size_t>(bh) * a.nchunk + chunk) * a.D + d;
     a.ksum[o] = sum;
@@ -351,22 +424,36 @@ __global__ void prologue_finalize_kernel(PrologueArgs a) {
 }
 
 // Pass 2: quantise.  Q, K: rotate (K also smoothed), per-token scale and codes.
-// V: per-channel codes, column sums per key block.  Each thread loads the next
-// token's Q, K, V and position before working on the current one; Q and K share
-// the RoPE coefficients of the token.  Column sums are kept per thread while a
-// warp stays in one key block, then combined across the warp's tokens and
-// added to shared memory.
+// V: per-channel codes, column sums per key block.  Q and K of a token share
+// the RoPE coefficients; column sums are kept per thread while a warp stays in
+// one key block, then combined across the warp's tokens and added to shared
+// memory.
 template <bool kBf16>
 __global__ void __launch_bounds__(kThreads, 3) prologue_quant_kernel(PrologueArgs a) {
+  using IO = StageIO<kBf16, 3>;
   __shared__ float rows[kThreads / 32][4][128];
   __shared__ int csum[kChunk / 16][128];
+  __shared__ uint64_t full[kStg];
+  __shared__ int abort_flag;
+  extern __shared__ __align__(128) uint8_t stg[];
   const int bh = blockIdx.y, chunk = blockIdx.x;
   const int lpt = a.D >> 3, tpw = 32 / lpt;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tok_in_warp = lane / lpt, c0 = (lane % lpt) * 8;
-  const int step = (kThreads / 32) * tpw, iters = kChunk / step;
+  const int step = (kThreads / 32) * tpw;
   const int nblk = kChunk / a.block_k;
+  const int n0 = chunk * kChunk;
+  const size_t head = static_cast<size_t>(bh) * a.N * a.D;
+  const size_t head4 = static_cast<size_t>(bh) * a.N * (a.D / 2);
+  const void* src[3] = {a.q, a.k, a.v};
+  RopePlan rp;
+  rp.init(a.s, c0);
   for (int i = threadIdx.x; i < nblk * a.D; i += kThreads) csum[i / a.D][i % a.D] = 0;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStg; ++s) mbar_init(full + s, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
   float kmean[8], vinv[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
@@ -374,25 +461,10 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_quant_kernel(PrologueArg
     vinv[i] = a.vinv[bh * a.D + c0 + i];
   }
   __syncthreads();
-  const int n0 = chunk * kChunk;
-  const size_t head = static_cast<size_t>(bh) * a.N * a.D;
-  const size_t head4 = static_cast<size_t>(bh) * a.N * (a.D / 2);
-  int n = n0 + warp * tpw + tok_in_warp;
-  Raw8<kBf16> rq{}, rk{}, rv{};
-  int gp[3] = {0, 0, 0};
-  auto fetch = [&](int nn) {
-    if (nn < a.N) {
-      const size_t o = head + static_cast<size_t>(nn) * a.D + c0;
-      load_raw8<kBf16>(a.q, o, rq);
-      load_raw8<kBf16>(a.k, o, rk);
-      load_raw8<kBf16>(a.v, o, rv);
-#pragma unroll
-      for (int j = 0; j < 3; ++j) gp[j] = __ldg(a.pos + 3 * nn + j);
-    }
-  };
-  fetch(n);
+  if (threadIdx.x == 0)
+    for (int sc = 0; sc < kStg; ++sc) IO::issue(src, head, a.D, a.N, n0, sc, stg, full);
   int cacc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-  int cblk = (warp * tpw) / a.block_k;  // key block of this warp's tokens in iteration 0
+  int cblk = (warp * tpw) / a.block_k;  // key block of this warp's first tokens
   // Adds this warp's per-thread column sums of block cblk to shared memory:
   // lanes holding the same channels (lpt apart) are combined first.
   auto flush = [&]() {
@@ -407,61 +479,74 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_quant_kernel(PrologueArg
 #pragma unroll
     for (int i = 0; i < 8; ++i) cacc[i] = 0;
   };
-  for (int it = 0; it < iters; ++it) {
-    const bool ok = n < a.N;
-    const int ncur = n;
-    const Raw8<kBf16> cq = rq, ck = rk, cv = rv;
-    const int g3[3] = {gp[0], gp[1], gp[2]};
-    n += step;
-    if (it + 1 < iters) fetch(n);
-    const int blk = (it * step + warp * tpw) / a.block_k;  // the same for the warp's tokens
-    if (blk != cblk) {
-      flush();
-      cblk = blk;
-    }
-    float xq[8], xk[8], xv[8], ca[4], cb[4];
-    if (ok) {
-      unpack8<kBf16>(cq, xq);
-      unpack8<kBf16>(ck, xk);
-      unpack8<kBf16>(cv, xv);
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) { xq[i] = 0.0f; xk[i] = 0.0f; xv[i] = 0.0f; }
-    }
-    const int z3[3] = {0, 0, 0};
-    rope_coef8(a.s, a.tab_a, a.tab_b, ok ? g3 : z3, c0, ca, cb);
-    rope_apply8(a.s, a.rot, ca, cb, c0, xq, rows[warp][tok_in_warp]);
-    rope_apply8(a.s, a.rot, ca, cb, c0, xk, rows[warp][tok_in_warp]);
-    float mq = 0.0f, mk = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      xk[i] = __fsub_rn(xk[i], kmean[i]);
-      mq = fmaxf(mq, fabsf(xq[i]));
-      mk = fmaxf(mk, fabsf(xk[i]));
-    }
-    mq = group_max(mq, lpt);
-    mk = group_max(mk, lpt);
-    int cq8[8], ck8[8], cv8[8];
-    const float iq = mq == 0.0f ? 0.0f : __fdiv_rn(7.0f, mq);
-    const float ik = mk == 0.0f ? 0.0f : __fdiv_rn(7.0f, mk);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      cq8[i] = quant4(xq[i], iq);
-      ck8[i] = quant4(xk[i], ik);
-      cv8[i] = quant4(xv[i], vinv[i]);
-    }
-    if (ok) {
-      const size_t o4 = head4 + static_cast<size_t>(ncur) * (a.D / 2) + (c0 >> 1);
-      *reinterpret_cast<uint32_t*>(a.q4 + o4) = pack8(cq8);
-      *reinterpret_cast<uint32_t*>(a.k4 + o4) = pack8(ck8);
-      *reinterpret_cast<uint32_t*>(a.v4 + o4) = pack8(cv8);
-      if (c0 == 0) {
-        a.sq[static_cast<size_t>(bh) * a.N + ncur] = __fdiv_rn(mq, 7.0f);
-        a.sk[static_cast<size_t>(bh) * a.N + ncur] = __fdiv_rn(mk, 7.0f);
+  bool ok = true;
+  for (int sc = 0; sc < kChunk / kSub && ok; ++sc) {
+    const int s = sc % kStg;
+    if (!(ok = stage_wait(full + s, (sc / kStg) & 1, &abort_flag))) break;
+    for (int ti = warp * tpw + tok_in_warp; ti - tok_in_warp < kSub; ti += step) {
+      const int n = n0 + sc * kSub + ti;
+      const bool valid = n < a.N;
+      const int blk = (sc * kSub + ti - tok_in_warp) / a.block_k;  // the same for the warp's tokens
+      if (blk != cblk) {
+        flush();
+        cblk = blk;
       }
+      float xq[8], xk[8], xv[8], ca[4], cb[4];
+      int gp[3] = {0, 0, 0};
+      if (valid) {
+        Raw8<kBf16> rq, rk, rv;
+        IO::read(stg, a.D, s, 0, ti, c0, rq);
+        IO::read(stg, a.D, s, 1, ti, c0, rk);
+        IO::read(stg, a.D, s, 2, ti, c0, rv);
+        unpack8<kBf16>(rq, xq);
+        unpack8<kBf16>(rk, xk);
+        unpack8<kBf16>(rv, xv);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) cacc[i] += cv8[i];
+        for (int j = 0; j < 3; ++j) gp[j] = __ldg(a.pos + 3 * n + j);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) { xq[i] = 0.0f; xk[i] = 0.0f; xv[i] = 0.0f; }
+      }
+      rope_coef8p(a.s, rp, a.tab_a, a.tab_b, gp, ca, cb);
+      rope_apply8(a.s, a.rot, ca, cb, c0, xq, rows[warp][tok_in_warp]);
+      rope_apply8(a.s, a.rot, ca, cb, c0, xk, rows[warp][tok_in_warp]);
+      float mq = 0.0f, mk = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        xk[i] = __fsub_rn(xk[i], kmean[i]);
+        mq = fmaxf(mq, fabsf(xq[i]));
+        mk = fmaxf(mk, fabsf(xk[i]));
+      }
+      mq = group_max(mq, lpt);
+      mk = group_max(mk, lpt);
+      uint32_t bq[8], bk[8], bv[8];
+      const float iq = mq == 0.0f ? 0.0f : __fdiv_rn(7.0f, mq);
+      const float ik = mk == 0.0f ? 0.0f : __fdiv_rn(7.0f, mk);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        bq[i] = quant4_bits(xq[i], iq);
+        bk[i] = quant4_bits(xk[i], ik);
+        bv[i] = quant4_bits(xv[i], vinv[i]);
+      }
+      if (valid) {
+        const size_t o4 = head4 + static_cast<size_t>(n) * (a.D / 2) + (c0 >> 1);
+        *reinterpret_cast<uint32_t*>(a.q4 + o4) = pack8_bits(bq);
+        *reinterpret_cast<uint32_t*>(a.k4 + o4) = pack8_bits(bk);
+        *reinterpret_cast<uint32_t*>(a.v4 + o4) = pack8_bits(bv);
+        if (c0 == 0) {
+          a.sq[static_cast<size_t>(bh) * a.N + n] = __fdiv_rn(mq, 7.0f);
+          a.sk[static_cast<size_t>(bh) * a.N + n] = __fdiv_rn(mk, 7.0f);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) cacc[i] += static_cast<int>(bv[i] - 0x4B400000u);
+      }
     }
+    __syncthreads();  // stage s consumed
+    if (threadIdx.x == 0 && sc + kStg < kChunk / kSub) IO::issue(src, head, a.D, a.N, n0, sc + kStg, stg, full);
+  }
+  if (!ok) {
+    if (threadIdx.x == 0) atomicOr(&g_prologue_status, kStatusTimeout);
+    return;
   }
   flush();
   __syncthreads();
@@ -542,6 +627,11 @@ WorkspaceLayout workspace_layout(const ra_problem& p) {
   return w;
 }
 
+template <typename K>
+static cudaError_t set_smem(K kern, int bytes) {
+  return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
 static cudaError_t launch_tables(const ra_problem& p, int rot, float* ta, float* tb, cudaStream_t st) {
   const SegInfo s = seg_info(p);
   const int T = static_cast<int>(rope_table_len(p));
@@ -570,13 +660,28 @@ cudaError_t launch_prologue(const ra_problem& p, int dtype, const void* q, const
   cudaError_t e = launch_tables(p, p.rot, const_cast<float*>(a.tab_a), const_cast<float*>(a.tab_b), st);
   if (e != cudaSuccess) return e;
   const dim3 grid(a.nchunk, p.B * p.H);
-  if (dtype == 1) prologue_reduce_kernel<true><<<grid, kThreads, 0, st>>>(a);
-  else prologue_reduce_kernel<false><<<grid, kThreads, 0, st>>>(a);
+  // Dynamic shared memory: kStg staged sub-chunks (the reduce pass reuses it
+  // for its per-thread partial sums, 12 bytes x 8 channels x threads).
+  const int el = dtype == 1 ? 2 : 4;
+  const int red_bytes = kStg * 2 * kSub * p.D * el > kThreads * 8 * 12 ? kStg * 2 * kSub * p.D * el : kThreads * 8 * 12;
+  const int quant_bytes = kStg * 3 * kSub * p.D * el;
+  if (dtype == 1) {
+    if ((e = set_smem(prologue_reduce_kernel<true>, red_bytes)) != cudaSuccess) return e;
+    prologue_reduce_kernel<true><<<grid, kThreads, red_bytes, st>>>(a);
+  } else {
+    if ((e = set_smem(prologue_reduce_kernel<false>, red_bytes)) != cudaSuccess) return e;
+    prologue_reduce_kernel<false><<<grid, kThreads, red_bytes, st>>>(a);
+  }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   prologue_finalize_kernel<<<p.B * p.H, 128, 0, st>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if (dtype == 1) prologue_quant_kernel<true><<<grid, kThreads, 0, st>>>(a);
-  else prologue_quant_kernel<false><<<grid, kThreads, 0, st>>>(a);
+  if (dtype == 1) {
+    if ((e = set_smem(prologue_quant_kernel<true>, quant_bytes)) != cudaSuccess) return e;
+    prologue_quant_kernel<true><<<grid, kThreads, quant_bytes, st>>>(a);
+  } else {
+    if ((e = set_smem(prologue_quant_kernel<false>, quant_bytes)) != cudaSuccess) return e;
+    prologue_quant_kernel<false><<<grid, kThreads, quant_bytes, st>>>(a);
+  }
   return cudaGetLastError();
 }
 
