@@ -138,6 +138,23 @@ def cpu_baseline(wl, target_s: float = 15.0, x=None):
                       f"attention of {rows} query rows over all {wl.N} keys; {t:.1f} s of CPU time"}
 
 
+def max_over_ranks(value: float, device) -> float:
+    """The largest of every rank's value (all ranks call this in the same
+    order); with one rank, the value itself."""
+    import torch
+    if not (torch.distributed.is_available() and torch.distributed.is_initialized()):
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(world: int, ops_per_rank: float, ms_per_step: float) -> float:
+    """Whole-job TOPS: every rank runs its own batch of ops_per_rank per step,
+    and the step takes the slowest rank's time."""
+    return world * ops_per_rank / (ms_per_step * 1e-3) / 1e12
+
+
 def _attn_traffic():
     """DRAM bytes per attention launch from the committed ncu summary, or None
     when the attention kernel's sources changed since those counters were taken."""
@@ -219,10 +236,7 @@ def run_ours(args, rank, world, local_rank):
     status = ra.sync_status()
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed region")
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dev)
 
     # end to end through the public API with host buffers: H2D of Q/K/V (pinned),
     # prologue + attention, D2H of the output, every step
@@ -244,11 +258,7 @@ def run_ours(args, rank, world, local_rank):
         out_h.copy_(out, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1) / args.steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
     h2d = sum(host[n].numel() * 2 for n in ("q", "k", "v")) + pos_h.numel() * 4
     d2h = out_h.numel() * 2
 
@@ -275,7 +285,7 @@ def run_ours(args, rank, world, local_rank):
 
     ops = wl.attn_ops()
     ms_step = total_ms / args.steps
-    value = world * ops / (ms_step * 1e-3) / 1e12
+    value = weak_scaling_value(world, ops, ms_step)
     pk = _peaks()
     int8_peak = 2.0 * pk["bf16_tflops"]        # nominal dense int8 / bf16 ratio on B200 = 2
     att_med = statistics.median(att_ms)
@@ -287,7 +297,7 @@ def run_ours(args, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "int4", "data": "synthetic (seeded, outlier-structured; no model weights)",
         "config": _config(wl, {"parallelism": f"independent batch per GPU x{world}"}),
-        "e2e": {"value": round(world * ops / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TOPS",
+        "e2e": {"value": round(weak_scaling_value(world, ops, e2e_ms), 2), "unit": "TOPS",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "roofline": {"bound": "tensor", "kernel": "attn_int4_kernel", "achieved": round(achieved, 1),
                      "peak": round(int8_peak, 1), "unit": "TFLOP/s", "frac": round(achieved / int8_peak, 4),
