@@ -20,7 +20,13 @@ _lib = None
 class OrcProblem(C.Structure):
     _fields_ = [("B", C.c_int), ("H", C.c_int), ("N", C.c_int), ("D", C.c_int),
                 ("seg", C.c_int * 3), ("grid", C.c_int * 3), ("theta", C.c_double),
-                ("rot", C.c_int), ("block_q", C.c_int), ("block_k", C.c_int)]
+                ("rot", C.c_int), ("block_q", C.c_int), ("block_k", C.c_int),
+                ("p_mode", C.c_int), ("l_mode", C.c_int)]
+
+
+# Ablation switches of the attention (reading R11 in ra_oracle.c).
+P_RANGE, P_LOCAL, P_SYMMETRIC = 0, 1, 2
+L_CODES, L_FP32 = 0, 1
 
 
 def lib():
@@ -34,6 +40,7 @@ def lib():
         _lib.orc_rope_rotate.argtypes = [P(OrcProblem), vp, vp, vp, C.c_int]
         _lib.orc_prologue_head.argtypes = [P(OrcProblem)] + [vp] * 14
         _lib.orc_p_code.argtypes = [C.c_float, C.c_float]
+        _lib.orc_p_code_sym.argtypes = [C.c_float, C.c_float]
         _lib.orc_attention_int4_rows.argtypes = [P(OrcProblem)] + [vp] * 7 + [C.c_int, C.c_int] + [vp] * 5
         _lib.orc_attention_int4_rows_given_codes.argtypes = [P(OrcProblem)] + [vp] * 8 + [C.c_int, C.c_int, vp, vp]
         _lib.orc_attention_exact_blocked_rows.argtypes = [P(OrcProblem), vp, vp, vp, C.c_int, C.c_int, vp, vp]
@@ -44,7 +51,7 @@ def lib():
 
 
 def problem(wl=None, *, N=None, D=None, seg=None, grid=None, theta=10000.0, rot=1,
-            block_q=128, block_k=64, B=1, H=1) -> OrcProblem:
+            block_q=128, block_k=64, B=1, H=1, p_mode=P_RANGE, l_mode=L_CODES) -> OrcProblem:
     """Build the C problem struct from a synth.inputs.Workload or keywords."""
     if wl is not None:
         B, H, D, seg, grid = wl.B, wl.H, wl.D, wl.seg, wl.grid
@@ -57,6 +64,7 @@ def problem(wl=None, *, N=None, D=None, seg=None, grid=None, theta=10000.0, rot=
     p.seg[:] = list(seg)
     p.grid[:] = list(grid)
     p.theta, p.rot, p.block_q, p.block_k = float(theta), int(rot), int(block_q), int(block_k)
+    p.p_mode, p.l_mode = int(p_mode), int(l_mode)
     return p
 
 
@@ -119,6 +127,10 @@ def prologue_head(p: OrcProblem, q: np.ndarray, k: np.ndarray, v: np.ndarray, po
 
 def p_code(S: float, m: float) -> int:
     return int(lib().orc_p_code(C.c_float(S), C.c_float(m)))
+
+
+def p_code_sym(S: float, m: float) -> int:
+    return int(lib().orc_p_code_sym(C.c_float(S), C.c_float(m)))
 
 
 def attention_int4_rows(p: OrcProblem, h: Dict[str, np.ndarray], row0: int, row1: int,

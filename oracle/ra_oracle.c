@@ -37,6 +37,12 @@
  *   R8 Keys past N in the last block do not take part (S = -inf, code -8,
  *      V = 0, excluded from colsum).
  *   R9 S = ((float)S_int * s_k[j]) * (s_q[i] * (1/sqrt(D))) in fp32.
+ *   R11 Ablation switches (off by default): p_mode LOCAL takes the codes of
+ *      a block against that block's own maximum and weights the block by
+ *      exp(m_block - m) in the recurrence; p_mode SYMMETRIC uses the
+ *      SageAttention-style codes c = rint(7 exp(S - m)) in [0, 7] with no zero
+ *      point, dequantised as c / 7; l_mode FP32 makes the denominator the
+ *      plain sum of exp(S - m_codes) instead of the dequantised code sum.
  *   R10 Codes are packed two per byte, element 2t in the low nibble, as
  *      4-bit two's complement.
  */
@@ -55,9 +61,13 @@ typedef struct {
   double theta;   /* RoPE base */
   int rot;        /* 0 = RoPE only, 1 = interleaved rotation, 2 = half rotation */
   int block_q, block_k;
+  int p_mode;     /* ORC_P_RANGE (default), ORC_P_LOCAL, ORC_P_SYMMETRIC (R11) */
+  int l_mode;     /* ORC_L_CODES (default), ORC_L_FP32 (R11) */
 } orc_problem;
 
 enum { ORC_OK = 0, ORC_BAD = 1 };
+enum { ORC_P_RANGE = 0, ORC_P_LOCAL = 1, ORC_P_SYMMETRIC = 2 };
+enum { ORC_L_CODES = 0, ORC_L_FP32 = 1 };
 
 static int seg_off(const orc_problem* p, int j) {
   int o = 0;
@@ -74,6 +84,8 @@ static int check_problem(const orc_problem* p) {
   }
   if (p->grid[0] * p->grid[1] * p->grid[2] < 1) return ORC_BAD;
   if (p->rot < 0 || p->rot > 2 || p->block_k < 1) return ORC_BAD;
+  if (p->p_mode < ORC_P_RANGE || p->p_mode > ORC_P_SYMMETRIC) return ORC_BAD;
+  if (p->l_mode < ORC_L_CODES || p->l_mode > ORC_L_FP32) return ORC_BAD;
   return ORC_OK;
 }
 
@@ -324,6 +336,21 @@ int orc_p_code(float S, float m) {
 }
 
 /*
+ * Symmetric P code of the SageAttention-style baseline that the pages compare
+ * against (papernotes page, key design 2: only the levels 0..7 of the signed
+ * range are used): c = round(7 P) in [0, 7], P = exp(S - m), no zero point.
+ * Same precision rules as orc_p_code.
+ */
+int orc_p_code_sym(float S, float m) {
+  if (isinf(S) && S < 0) return 0;
+  double e = exp((double)S - (double)m);
+  double r = rint(7.0 * e);
+  if (r < 0.0) r = 0.0;
+  if (r > 7.0) r = 7.0;
+  return (int)r;
+}
+
+/*
  * Blocked attention of rows [row0, row1) of one head with online softmax
  * (papernotes page: "overall framework" flowchart D-F, key design 2; the
  * FlashAttention recurrence with the running ("sliding") row maximum).
@@ -332,6 +359,11 @@ int orc_p_code(float S, float m) {
  *   orc_p_code against the running max m_t after block t (R6),
  *   acc_t[d] = sum_j c_ij v4_jd + 8 colsum_t[d] (the zero-point correction),
  *   O <- alpha O + (s_v/15) acc_t, l <- alpha l + lq_t/15 (R7).
+ *   With the R11 switches: the codes are taken against m_c (the block's own
+ *   maximum for LOCAL, else m_t) and the block enters with the weight
+ *   beta = exp(m_c - m_t); SYMMETRIC codes have 7 levels and no zero point
+ *   (acc_t = sum_j c_ij v4_jd, scale s_v/7, lq_t/7); FP32 replaces lq_t/L by
+ *   sum_j exp(S_ij - m_c).
  * quant == 0: the same recurrence on fp64 inputs qf/kf/vf with
  *   S = q.k / sqrt(D) and P = exp(S - m) (no quantisation) -- used by the
  *   tests to show that the blocked recurrence equals plain softmax attention.
@@ -372,7 +404,7 @@ static void attn_row(const orc_problem* p, const orc_attn_in* in, int quant, int
     int j0 = t * Bk, j1 = j0 + Bk < N ? j0 + Bk : N;
     double alpha;
     if (quant) {
-      float mt = m;
+      float mt = m, mb = -INFINITY;
       for (int j = j0; j < j1; ++j) {
         const uint8_t* kr = in->k4 + (size_t)j * (D / 2);
         int32_t sint = 0;
@@ -381,27 +413,36 @@ static void attn_row(const orc_problem* p, const orc_attn_in* in, int quant, int
         float v = (float)sint * in->sk[j];
         S[j - j0] = v * ci;
         if (S[j - j0] > mt) mt = S[j - j0];
+        if (S[j - j0] > mb) mb = S[j - j0];
       }
       alpha = (m == -INFINITY) ? 0.0 : exp((double)m - (double)mt);
       m = mt;
+      const int sym = p->p_mode == ORC_P_SYMMETRIC;
+      const float mc = p->p_mode == ORC_P_LOCAL ? mb : m;   /* the max the codes use */
+      const double beta = exp((double)mc - (double)m);      /* 1 unless LOCAL */
+      const int zp = sym ? 0 : 8;
+      const double levels = sym ? 7.0 : 15.0;
       int lq = 0;
+      double le = 0.0;
       for (int d = 0; d < D; ++d) acc[d] = 0.0;
       int32_t acci[256];
       for (int d = 0; d < D; ++d) acci[d] = 0;
       for (int j = j0; j < j1; ++j) {
-        int c = in->codes_in ? in->codes_in[(size_t)(i - in->row0) * N + j] : orc_p_code(S[j - j0], m);
+        int c = in->codes_in ? in->codes_in[(size_t)(i - in->row0) * N + j]
+                             : (sym ? orc_p_code_sym(S[j - j0], mc) : orc_p_code(S[j - j0], mc));
         if (c_dump) c_dump[j] = (int8_t)c;
-        lq += c + 8;
+        lq += c + zp;
+        le += exp((double)S[j - j0] - (double)mc);
         const uint8_t* vr = in->v4 + (size_t)j * (D / 2);
         for (int d = 0; d < D; ++d) acci[d] += c * unpack4(vr, d);
       }
       for (int d = 0; d < D; ++d) {
-        acci[d] += 8 * in->colsum[(size_t)t * D + d];
+        acci[d] += zp * in->colsum[(size_t)t * D + d];
         if (acc_dump) acc_dump[(size_t)t * D + d] = acci[d];
-        acc[d] = (double)in->sv[d] / 15.0 * (double)acci[d];
+        acc[d] = (double)in->sv[d] / levels * (double)acci[d];
       }
-      for (int d = 0; d < D; ++d) O[d] = alpha * O[d] + acc[d];
-      l = alpha * l + (double)lq / 15.0;
+      for (int d = 0; d < D; ++d) O[d] = alpha * O[d] + beta * acc[d];
+      l = alpha * l + beta * (p->l_mode == ORC_L_FP32 ? le : (double)lq / levels);
     } else {
       double mt = md;
       for (int j = j0; j < j1; ++j) {

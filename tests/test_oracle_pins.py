@@ -403,3 +403,132 @@ def test_given_codes_entry(orc):
     assert np.abs(flipped[i] - expect).max() <= 1e-12 * np.abs(expect).max()
     others = np.arange(R) != i
     assert np.array_equal(flipped[others], r["out"][others])
+
+
+# --- ablation switches (reading R11): block-local max, symmetric P, fp32 l ---
+
+def _brute_force_modes(wl, h, rows, p_mode, l_mode):
+    """Unblocked closed form of the INT4 path under the ablation switches.
+
+    Key j of block t(j) is coded against M_c = the block's own maximum (LOCAL)
+    or the running maximum after its block (otherwise); its weight relative to
+    the final maximum is exp(M_c - M_final).  Range codes are rint(15 e) - 8
+    dequantised as (c + 8) / 15, symmetric codes rint(7 e) dequantised as c / 7,
+    e = exp(S - M_c).  Output = sum_j w_j P_j s_v v_j / sum_j w_j L_j with
+    P_j the dequantised code and L_j = P_j (code denominator) or e_j (fp32)."""
+    from oracle import P_LOCAL, P_SYMMETRIC, L_FP32, unpack_codes
+    N, D, Bk = wl.N, wl.D, wl.block_k
+    q = unpack_codes(h["q4"]).astype(np.int64)
+    k = unpack_codes(h["k4"]).astype(np.int64)
+    v = unpack_codes(h["v4"]).astype(np.float64) * h["sv"].astype(np.float64)
+    ci = np.float32(h["sq"][rows]) * np.float32(1.0 / math.sqrt(D))
+    S = ((q[rows] @ k.T).astype(np.float32) * h["sk"][None, :].astype(np.float32)) * ci[:, None]
+    nb = -(-N // Bk)
+    bmax = np.stack([S[:, t * Bk:(t + 1) * Bk].max(axis=1) for t in range(nb)], axis=1)
+    run = np.maximum.accumulate(bmax, axis=1)
+    Mc = np.repeat(bmax if p_mode == P_LOCAL else run, Bk, axis=1)[:, :N].astype(np.float64)
+    e = np.exp(S.astype(np.float64) - Mc)
+    if p_mode == P_SYMMETRIC:
+        codes = np.rint(7.0 * e)
+        deq = codes / 7.0
+    else:
+        codes = np.rint(15.0 * e) - 8
+        deq = (codes + 8) / 15.0
+    w = np.exp(Mc - run[:, -1:].astype(np.float64))
+    den = (w * (e if l_mode == L_FP32 else deq)).sum(axis=1, keepdims=True)
+    return ((w * deq) @ v) / den, codes
+
+
+@pytest.mark.parametrize("name", ["tiny", "small"])
+@pytest.mark.parametrize("p_mode,l_mode", [(0, 1), (1, 0), (1, 1), (2, 0), (2, 1)])
+def test_ablation_switches_equal_unblocked_brute_force(orc, name, p_mode, l_mode):
+    wl, _, x, h = _head(orc, name)
+    p = orc.problem(wl, p_mode=p_mode, l_mode=l_mode)
+    rows = np.arange(min(wl.N, 96))
+    r = orc.attention_int4_rows(p, h, 0, len(rows), dumps=True)
+    ref, codes = _brute_force_modes(wl, h, rows, p_mode, l_mode)
+    assert np.array_equal(r["codes"], codes.astype(np.int8))
+    assert np.abs(r["out"] - ref).max() <= 1e-12 * np.abs(ref).max()
+
+
+def test_brute_force_modes_reduce_to_the_range_path(orc):
+    """The generalised closed form, switches off, is the range-rectified one."""
+    wl, p, x, h = _head(orc, "small")
+    rows = np.arange(64)
+    a, ca = _brute_force_modes(wl, h, rows, 0, 0)
+    b, cb = _brute_force_quantised(wl, h, rows)
+    assert np.array_equal(ca, cb) and np.abs(a - b).max() <= 1e-14 * np.abs(b).max()
+
+
+def test_local_max_with_one_block_is_the_running_max(orc):
+    """With a single key block the block maximum is the running maximum."""
+    wl, _, x, h = _head(orc, "tiny")
+    for l_mode in (0, 1):
+        pb, pl = orc.problem(wl, l_mode=l_mode), orc.problem(wl, p_mode=1, l_mode=l_mode)
+        pb.block_k = pl.block_k = wl.N
+        base = orc.attention_int4_rows(pb, h, 0, wl.N, dumps=True)
+        loc = orc.attention_int4_rows(pl, h, 0, wl.N, dumps=True)
+        assert np.array_equal(base["codes"], loc["codes"])
+        assert np.array_equal(base["out"], loc["out"]) and np.array_equal(base["lse"], loc["lse"])
+
+
+def test_local_max_codes_differ_and_reach_seven_in_every_block(orc):
+    """Against its own maximum every block has a key with P = 1 (code 7)."""
+    wl, _, x, h = _head(orc, "small")
+    r = orc.attention_int4_rows(orc.problem(wl, p_mode=1), h, 0, 32, dumps=True)
+    base = orc.attention_int4_rows(orc.problem(wl), h, 0, 32, dumps=True)
+    assert not np.array_equal(r["codes"], base["codes"])
+    Bk = wl.block_k
+    for t in range(0, wl.N, Bk):
+        assert (r["codes"][:, t:t + Bk].max(axis=1) == 7).all()
+
+
+def test_symmetric_codes_use_levels_zero_to_seven(orc):
+    """SageAttention-style P: rint(7 P), levels 0..7 only, P = 1 -> 7, P -> 0 -> 0."""
+    assert orc.p_code_sym(2.0, 2.0) == 7
+    assert orc.p_code_sym(-40.0, 0.0) == 0 and orc.p_code_sym(float("-inf"), 0.0) == 0
+    for seven_p, code in ((3.6, 4), (3.4, 3), (1.4, 1), (0.55, 1), (0.45, 0), (6.6, 7)):
+        assert orc.p_code_sym(float(np.float32(math.log(seven_p / 7))), 0.0) == code, seven_p
+    wl, _, x, h = _head(orc, "small")
+    r = orc.attention_int4_rows(orc.problem(wl, p_mode=2), h, 0, wl.N, dumps=True)
+    assert np.unique(r["codes"]).tolist() == list(range(0, 8))
+
+
+def test_symmetric_acc_has_no_zero_point(orc):
+    wl, _, x, h = _head(orc, "small")
+    r = orc.attention_int4_rows(orc.problem(wl, p_mode=2), h, 0, 64, dumps=True)
+    v = orc.unpack_codes(h["v4"]).astype(np.int64)
+    c = r["codes"].astype(np.int64)
+    Bk = wl.block_k
+    for t in range(-(-wl.N // Bk)):
+        sl = slice(t * Bk, (t + 1) * Bk)
+        assert np.array_equal(r["acc"][:, t], c[:, sl] @ v[sl])
+
+
+def test_uniform_row_gives_the_mean_of_v_in_every_mode(orc):
+    """A zero query row has S = 0 for every key: every mode gives the mean of
+    the dequantised V and lse = ln N (fp32 l) or ln(N * 15 / 15) = ln N."""
+    wl, _, x, h = _head(orc, "small")
+    h = dict(h)
+    h["q4"] = h["q4"].copy()
+    h["sq"] = h["sq"].copy()
+    h["q4"][3] = 0          # what the prologue emits for an all-zero query token
+    h["sq"][3] = 0.0
+    mean = (orc.unpack_codes(h["v4"]).astype(np.float64) * h["sv"].astype(np.float64)).mean(axis=0)
+    for p_mode in (0, 1, 2):
+        for l_mode in (0, 1):
+            r = orc.attention_int4_rows(orc.problem(wl, p_mode=p_mode, l_mode=l_mode), h, 3, 4)
+            assert np.abs(r["out"][0] - mean).max() <= 1e-12 * np.abs(mean).max(), (p_mode, l_mode)
+            assert abs(r["lse"][0] - math.log(wl.N)) <= 1e-12, (p_mode, l_mode)
+
+
+def test_fp32_l_changes_only_the_denominator(orc):
+    """Same codes and numerator: the two outputs of a row differ by one factor."""
+    wl, _, x, h = _head(orc, "small")
+    for p_mode in (0, 1, 2):
+        a = orc.attention_int4_rows(orc.problem(wl, p_mode=p_mode), h, 0, 64, dumps=True)
+        b = orc.attention_int4_rows(orc.problem(wl, p_mode=p_mode, l_mode=1), h, 0, 64, dumps=True)
+        assert np.array_equal(a["codes"], b["codes"])
+        ratio = np.exp(a["lse"] - b["lse"])          # l_codes / l_fp32
+        assert np.abs(b["out"] - a["out"] * ratio[:, None]).max() <= 1e-12 * np.abs(a["out"]).max()
+        assert np.all(ratio > 0) and not np.allclose(ratio, 1.0)
