@@ -31,6 +31,9 @@ if ROOT not in sys.path:
 
 METRIC = "INT4 attn TOPS (4N²DH/t) & % INT8 tensor peak at N=32760,H=40,D=128"
 KERNELS_PER_STEP = 5  # rope table, channel reduce, finalize, quantise, attention
+# (name, p_mode, l_mode) of the attention's ablation switches timed after the step.
+ABLATIONS = (("fp32_l", 0, 1), ("local_max", 1, 0), ("local_max_fp32_l", 1, 1),
+             ("symmetric_p", 2, 0), ("symmetric_p_fp32_l", 2, 1))
 
 
 def _peaks():
@@ -283,6 +286,28 @@ def run_ours(args, rank, world, local_rank):
     fb_ms = statistics.median(fb)
     del qr, kr, out_b
 
+    # The ablation switches of the attention (block-local max, symmetric P,
+    # fp32 denominator), each timed on its own on the same codes; not part of
+    # the INT4 step.
+    abl = {}
+    if wl.block_k == 64:
+        for name, pm, lm in ABLATIONS:
+            for _ in range(2):
+                ra.attn_int4(p, codes, out=out, p_mode=pm, l_mode=lm)
+            torch.cuda.synchronize(dev)
+            ts = []
+            for _ in range(max(3, args.steps // 8)):
+                a0 = torch.cuda.Event(enable_timing=True)
+                a1 = torch.cuda.Event(enable_timing=True)
+                a0.record(stream)
+                ra.attn_int4(p, codes, out=out, p_mode=pm, l_mode=lm)
+                a1.record(stream)
+                torch.cuda.synchronize(dev)
+                ts.append(a0.elapsed_time(a1))
+            if ra.sync_status() != 0:
+                raise RuntimeError(f"device status not ok after the {name} ablation")
+            abl[name] = statistics.median(ts)
+
     ops = wl.attn_ops()
     ms_step = total_ms / args.steps
     value = weak_scaling_value(world, ops, ms_step)
@@ -311,6 +336,8 @@ def run_ours(args, rank, world, local_rank):
         "bf16_fallback": {"ms": round(fb_ms, 4), "tflops": round(ops / (fb_ms * 1e-3) / 1e12, 1),
                           "peak": pk["bf16_tflops"], "frac": round(ops / (fb_ms * 1e-3) / 1e12 / pk["bf16_tflops"], 4),
                           "kernel": "attn_bf16_kernel", "note": "4N^2DH flops of bf16 attention on the RoPE'd inputs"},
+        "ablations": {n: {"ms": round(t, 4), "tops": round(ops / (t * 1e-3) / 1e12, 1),
+                          "frac": round(ops / (t * 1e-3) / 1e12 / int8_peak, 4)} for n, t in abl.items()},
         "gpu_launches": KERNELS_PER_STEP * args.steps,
         "clocks": clk.summary(),
     }

@@ -158,6 +158,48 @@ ra_status ra_test_int4_codes(const ra_problem* p,
                              void* out, float* lse, void* stream);
 
 /*
+ * Ablation switches of the INT4 attention.  The method's choices (papernotes
+ * page, key design 2) are the defaults; the alternatives it is compared with
+ * can be measured with the same kernels:
+ *   p_mode  RA_P_RANGE      range-rectified codes against the running maximum
+ *                           (default, as ra_attn_int4);
+ *           RA_P_LOCAL_MAX  the same codes against each key block's own
+ *                           maximum; block t then enters the output and the
+ *                           denominator with the weight exp(m_block - m);
+ *           RA_P_SYMMETRIC  SageAttention-style codes c = rint(7 exp(S - m))
+ *                           in [0, 7] (levels 0..7 only), no zero point:
+ *                           acc = sum_j c_ij v4[j, d], dequantised as c / 7.
+ *   l_mode  RA_L_CODES      denominator = sum of the dequantised codes (default);
+ *           RA_L_FP32       denominator = fp32 sum of exp(S - m_c), m_c the
+ *                           maximum the codes are taken against.
+ * opts == NULL selects the defaults.  A mode other than the defaults is
+ * implemented for block_k = 64 only (RA_ERR_UNSUPPORTED otherwise); an out of
+ * range mode is RA_ERR_INVALID_ARG.  All other arguments as ra_attn_int4 /
+ * ra_test_int4_codes; in the test entry p_dump holds the stored codes (c in
+ * [-8, 7], or [0, 7] for RA_P_SYMMETRIC) and acc_dump the accumulator
+ * sum_j (c_ij + zero point) v4[j, d].
+ */
+typedef enum { RA_P_RANGE = 0, RA_P_LOCAL_MAX = 1, RA_P_SYMMETRIC = 2 } ra_p_mode;
+typedef enum { RA_L_CODES = 0, RA_L_FP32 = 1 } ra_l_mode;
+typedef struct {
+  int p_mode;  /* ra_p_mode */
+  int l_mode;  /* ra_l_mode */
+} ra_attn_opts;
+
+ra_status ra_attn_int4_opts(const ra_problem* p, const ra_attn_opts* opts,
+                            const uint8_t* q4, const float* sq,
+                            const uint8_t* k4, const float* sk,
+                            const uint8_t* v4, const float* sv,
+                            void* out, float* lse, void* stream);
+ra_status ra_test_int4_codes_opts(const ra_problem* p, const ra_attn_opts* opts,
+                                  const uint8_t* q4, const float* sq,
+                                  const uint8_t* k4, const float* sk,
+                                  const uint8_t* v4, const float* sv,
+                                  int b, int h, int q_tile,
+                                  int32_t* s_dump, int8_t* p_dump, int32_t* acc_dump,
+                                  void* out, float* lse, void* stream);
+
+/*
  * 3D RoPE only (no rotation, no quantisation) of Q and K, output bf16: the
  * input of the bf16 fallback path (papernotes page, key design 3: sensitive
  * layers and steps keep full-precision attention; rotation does not change

@@ -17,11 +17,13 @@ import torch
 __all__ = [
     "ROT_NONE", "ROT_INTERLEAVED", "ROT_HALF", "RaError", "Problem", "lib", "workspace_bytes",
     "rope_rotate_quant", "attn_int4", "test_int4_codes", "rope_bf16", "attn_bf16_fallback",
-    "sync_status", "library_path",
+    "sync_status", "library_path", "AttnOpts", "P_RANGE", "P_LOCAL_MAX", "P_SYMMETRIC", "L_CODES", "L_FP32",
 ]
 
 ROT_NONE, ROT_INTERLEAVED, ROT_HALF = 0, 1, 2
 DT_F32, DT_BF16 = 0, 1
+P_RANGE, P_LOCAL_MAX, P_SYMMETRIC = 0, 1, 2   # ra_attn_opts.p_mode
+L_CODES, L_FP32 = 0, 1                        # ra_attn_opts.l_mode
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libra.so")
@@ -52,6 +54,15 @@ class Problem(C.Structure):
         return p
 
 
+class AttnOpts(C.Structure):
+    """ra_attn_opts: the ablation switches of the INT4 attention."""
+    _fields_ = [("p_mode", C.c_int), ("l_mode", C.c_int)]
+
+
+def _opts(p_mode: int, l_mode: int):
+    return None if (p_mode, l_mode) == (P_RANGE, L_CODES) else C.byref(AttnOpts(int(p_mode), int(l_mode)))
+
+
 def lib():
     """Loads libra.so; raises if it has not been built."""
     global _lib
@@ -67,11 +78,13 @@ def lib():
         L.ra_rope_rotate_quant.argtypes = [P, C.c_int] + [vp] * 13 + [sz, vp]
         L.ra_attn_int4.argtypes = [P] + [vp] * 9
         L.ra_test_int4_codes.argtypes = [P] + [vp] * 6 + [C.c_int] * 3 + [vp] * 6
+        L.ra_attn_int4_opts.argtypes = [P, vp] + [vp] * 9
+        L.ra_test_int4_codes_opts.argtypes = [P, vp] + [vp] * 6 + [C.c_int] * 3 + [vp] * 6
         L.ra_rope_bf16.argtypes = [P, C.c_int] + [vp] * 6 + [sz, vp]
         L.ra_attn_bf16_fallback.argtypes = [P] + [vp] * 6
         L.ra_sync_status.argtypes = [vp]
         for name in ("ra_rope_rotate_quant", "ra_attn_int4", "ra_test_int4_codes", "ra_rope_bf16",
-                     "ra_attn_bf16_fallback", "ra_sync_status"):
+                     "ra_attn_bf16_fallback", "ra_sync_status", "ra_attn_int4_opts", "ra_test_int4_codes_opts"):
             getattr(L, name).restype = C.c_int
         _lib = L
     return _lib
@@ -154,23 +167,26 @@ def rope_rotate_quant(p: Problem, q: torch.Tensor, k: torch.Tensor, v: torch.Ten
 
 
 def attn_int4(p: Problem, codes: Dict[str, torch.Tensor], out: Optional[torch.Tensor] = None,
-              lse: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """ra_attn_int4 on the prologue's outputs; returns out [B, H, N, D] bf16."""
+              lse: Optional[torch.Tensor] = None, stream=None, p_mode: int = P_RANGE,
+              l_mode: int = L_CODES) -> torch.Tensor:
+    """ra_attn_int4 (ra_attn_int4_opts for the ablation switches) on the
+    prologue's outputs; returns out [B, H, N, D] bf16."""
     B, H, N, D = p.B, p.H, p.N, p.D
     if out is None:
         out = torch.empty(B, H, N, D, dtype=torch.bfloat16, device=codes["q4"].device)
-    rc = lib().ra_attn_int4(
-        C.byref(p), _ptr(codes["q4"], torch.uint8, (B, H, N, D // 2)), _ptr(codes["sq"], torch.float32, (B, H, N)),
+    rc = lib().ra_attn_int4_opts(
+        C.byref(p), _opts(p_mode, l_mode), _ptr(codes["q4"], torch.uint8, (B, H, N, D // 2)), _ptr(codes["sq"], torch.float32, (B, H, N)),
         _ptr(codes["k4"], torch.uint8, (B, H, N, D // 2)), _ptr(codes["sk"], torch.float32, (B, H, N)),
         _ptr(codes["v4"], torch.uint8, (B, H, N, D // 2)), _ptr(codes["sv"], torch.float32, (B, H, D)),
         _ptr(out, torch.bfloat16, (B, H, N, D), "out"), _ptr(lse, torch.float32, (B, H, N), "lse"),
         C.c_void_p(_stream(stream)))
-    _check("ra_attn_int4", rc)
+    _check("ra_attn_int4_opts", rc)
     return out
 
 
-def test_int4_codes(p: Problem, codes: Dict[str, torch.Tensor], b: int, h: int, q_tile: int, stream=None):
-    """ra_test_int4_codes: returns (out, lse, s_dump, p_dump, acc_dump) for tile q_tile of head (b, h)."""
+def test_int4_codes(p: Problem, codes: Dict[str, torch.Tensor], b: int, h: int, q_tile: int, stream=None,
+                    p_mode: int = P_RANGE, l_mode: int = L_CODES):
+    """ra_test_int4_codes(_opts): returns (out, lse, s_dump, p_dump, acc_dump) for tile q_tile of head (b, h)."""
     B, H, N, D = p.B, p.H, p.N, p.D
     dev = codes["q4"].device
     out = torch.empty(B, H, N, D, dtype=torch.bfloat16, device=dev)
@@ -178,13 +194,13 @@ def test_int4_codes(p: Problem, codes: Dict[str, torch.Tensor], b: int, h: int, 
     s = torch.zeros(128, N, dtype=torch.int32, device=dev)
     pc = torch.zeros(128, N, dtype=torch.int8, device=dev)
     acc = torch.zeros(128, _nblocks(p), D, dtype=torch.int32, device=dev)
-    rc = lib().ra_test_int4_codes(
-        C.byref(p), _ptr(codes["q4"], torch.uint8), _ptr(codes["sq"], torch.float32),
+    rc = lib().ra_test_int4_codes_opts(
+        C.byref(p), _opts(p_mode, l_mode), _ptr(codes["q4"], torch.uint8), _ptr(codes["sq"], torch.float32),
         _ptr(codes["k4"], torch.uint8), _ptr(codes["sk"], torch.float32),
         _ptr(codes["v4"], torch.uint8), _ptr(codes["sv"], torch.float32),
         int(b), int(h), int(q_tile), _ptr(s), _ptr(pc), _ptr(acc), _ptr(out), _ptr(lse),
         C.c_void_p(_stream(stream)))
-    _check("ra_test_int4_codes", rc)
+    _check("ra_test_int4_codes_opts", rc)
     return out, lse, s, pc, acc
 
 

@@ -7,6 +7,10 @@
 //   acc_t = sum_j (c_ij + 8) v4_jd  (= sum_j c_ij v4_jd + 8 colsum_t: the
 //           zero-point correction folded into the integer accumulator)
 //   O = sum_t alpha-chain (s_v/15) acc_t / sum_t alpha-chain sum_j (c_ij+8)/15
+//   Ablation modes (the alternatives key design 2 is compared with): codes
+//   against each block's own maximum, weighted exp(m_block - m) (LOCAL);
+//   SageAttention-style codes rint(7 exp(S - m)) in [0, 7], no zero point
+//   (SYMMETRIC); the denominator as the fp32 sum of exp(S - m) (FP32 l).
 //
 // B200 design:
 //   * No 4-bit integer MMA exists on sm_100a; packed nibbles are widened to s8
@@ -189,7 +193,9 @@ __device__ __forceinline__ bool wait_at(uint64_t* bar, uint32_t parity, volatile
   return r > 0;
 }
 
-template <int D, int BN, bool DUMP>
+// MODE bits 0-1: P codes (0 range-rectified, 1 block-local maximum, 2
+// symmetric); bit 2: fp32 denominator.
+template <int D, int BN, bool DUMP, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const AttnParams prm) {
@@ -406,7 +412,11 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     // instruction, each rounded exactly like the scalar form).
     const float2 kNegMagic2 = make_float2(-kMagicF, -kMagicF);
     const float2 kMagic2 = make_float2(kMagicF, kMagicF);
-    const float2 k15x2 = make_float2(15.0f, 15.0f);
+    constexpr int kPMode = MODE & 3;
+    constexpr bool kLf = (MODE & 4) != 0;
+    constexpr float kLevels = kPMode == 2 ? 7.0f : 15.0f;  // code for P = 1
+    constexpr int kZero = kPMode == 2 ? 0 : 8;              // zero point of the stored codes
+    const float2 kLv2 = make_float2(kLevels, kLevels);
     uint32_t g = 0;
     bool ok = true;
     float2 F2[kFr / 2];  // F[2i], F[2i+1] of this thread's columns
@@ -476,6 +486,7 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       for (int q = 0; q < (kHD - kFr) / 4; ++q) Fs[q] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
       float m_run = -INFINITY, m_ref = 0.0f, w = 1.0f, Lf = 0.0f;
       int Lrun = 0;   // code sum of the row since the last fold (denominator)
+      float Lrun_e = 0.0f;  // fp32 sum of exp(S - m) since the last fold (fp32 denominator)
       int Labs = 0;   // code sum of the row since the last reset of A (magnitude bound)
       for (int t = 0; t < nb; ++t, ++g) {
         const uint32_t buf = g & 1;
@@ -513,17 +524,28 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const float m_blk = __fmul_rn(vmax, ci);
         const float m_new = fmaxf(m_run, m_blk);
         const bool grow = m_new > m_run;
-        const float Mp = __fmul_rn(m_new, kLog2e);
+        const float Mp = __fmul_rn(kPMode == 1 ? m_blk : m_new, kLog2e);  // the max the codes use
         const float2 nMp2 = make_float2(-Mp, -Mp);
         // P code c + 8 = rint(15 exp2(y)): adding 15 e to 1.5 * 2^23 rounds it
         // to an integer that lands in the low byte of the sum's bits.
         uint32_t words[kHK / 4];
+        float2 esum = make_float2(0.0f, 0.0f);
 #pragma unroll
         for (int q = 0; q < kHK / 4; ++q) {
           const float2 x01 = __ffma2_rn(v2[2 * q], cpi2, nMp2);
           const float2 x23 = __ffma2_rn(v2[2 * q + 1], cpi2, nMp2);
-          const float2 t01 = __ffma2_rn(k15x2, make_float2(ex2_approx(x01.x), ex2_approx(x01.y)), kMagic2);
-          const float2 t23 = __ffma2_rn(k15x2, make_float2(ex2_approx(x23.x), ex2_approx(x23.y)), kMagic2);
+          float2 e01 = make_float2(ex2_approx(x01.x), ex2_approx(x01.y));
+          float2 e23 = make_float2(ex2_approx(x23.x), ex2_approx(x23.y));
+          const float2 t01 = __ffma2_rn(kLv2, e01, kMagic2);
+          const float2 t23 = __ffma2_rn(kLv2, e23, kMagic2);
+          if constexpr (kLf) {
+            if (nvalid < BN) {  // keys past N (NaN scores) do not count
+              const int j = hh * kHK + 4 * q;
+              e01 = make_float2(j < nvalid ? e01.x : 0.0f, j + 1 < nvalid ? e01.y : 0.0f);
+              e23 = make_float2(j + 2 < nvalid ? e23.x : 0.0f, j + 3 < nvalid ? e23.y : 0.0f);
+            }
+            esum = __fadd2_rn(esum, __fadd2_rn(e01, e23));
+          }
           words[q] = __byte_perm(__byte_perm(__float_as_uint(t01.x), __float_as_uint(t01.y), 0x0040),
                                  __byte_perm(__float_as_uint(t23.x), __float_as_uint(t23.y), 0x0040), 0x5410);
         }
@@ -541,6 +563,11 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         for (int q = 0; q < kHK / 4; ++q) wsum += words[q];
         int lq = static_cast<int>(__dp4a(wsum, 0x01010101u, 0u));  // unsigned bytes
         lq += __shfl_xor_sync(0xFFFFFFFFu, lq, 16);
+        float le = 0.0f;
+        if constexpr (kLf) {
+          le = esum.x + esum.y;
+          le += __shfl_xor_sync(0xFFFFFFFFu, le, 16);
+        }
         // P codes over the S columns they came from: word q of half hh is
         // column hh * BN / 8 + q; P.V reads kKeysPV keys, those past BN are 0.
         tmem_st_h<kHK / 4, kHK / 4>(tS, words);
@@ -555,7 +582,7 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           for (int j = 0; j < kHK; ++j)
             if (hh * kHK + j < nvalid)
               prm.dump_p[static_cast<size_t>(r) * prm.N + t * BN + hh * kHK + j] =
-                  static_cast<int8_t>(((words[j >> 2] >> (8 * (j & 3))) & 0xFF) - 8);
+                  static_cast<int8_t>(((words[j >> 2] >> (8 * (j & 3))) & 0xFF) - kZero);
         }
         // Weight of the coming segment; a rescale moves the reference max.
         float w_new = w, sc = 1.0f;
@@ -572,12 +599,15 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             w_new = ex2_approx(x);
           }
         }
+        // Block-local codes: every block has its own weight exp(m_block - m_ref).
+        if constexpr (kPMode == 1) w_new = t == 0 ? 1.0f : ex2_approx(__fmul_rn(m_blk - m_ref, kLog2e));
+        const bool change = grow || (kPMode == 1 && w_new != w);
         // Fold when a row's maximum grows (its earlier codes used the old
         // maximum); reset A when its magnitude bound nears the exact range of
         // the read-back (|A| < 2^22).
         const bool near_bound = (Labs + 15 * BN) * 112 >= (1 << 22) - 4096;
         const bool reset = __any_sync(0xFFFFFFFFu, (t > 0) && (near_bound || DUMP));
-        if (reset || __any_sync(0xFFFFFFFFu, (t > 0) && grow)) {
+        if (reset || __any_sync(0xFFFFFFFFu, (t > 0) && change)) {
           if (!(ok = wait_at(B.pv_done + tt * 2 + ((g - 1) & 1), ((g - 1) >> 1) & 1, abort_flag, 12u, g))) break;
           __syncwarp();
           tc_fence_after();
@@ -593,13 +623,15 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             w *= sc;
           }
           fold(reset ? w : w - w_new, reset, t - 1, dump_tile);
-          Lf = fmaf(w, static_cast<float>(Lrun), Lf);
+          Lf = fmaf(w, kLf ? Lrun_e : static_cast<float>(Lrun), Lf);
           Lrun = 0;
+          Lrun_e = 0.0f;
           if (reset) Labs = 0;
         }
         w = w_new;
         Labs += lq;
         Lrun += lq;
+        Lrun_e += le;
         m_run = m_new;
         tc_fence_before();
         __syncwarp();
@@ -614,9 +646,11 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       __syncwarp();
       tc_fence_after();
       fold(w, true, nb - 1, dump_tile);
-      Lf = fmaf(w, static_cast<float>(Lrun), Lf);
+      Lf = fmaf(w, kLf ? Lrun_e : static_cast<float>(Lrun), Lf);
       if (row_ok) {
-        const float inv = 1.0f / (16.0f * Lf);
+        // O = (s_v / L) (acc / 16) / l with L the code levels; l is the code
+        // sum / L, or the fp32 sum of exp.
+        const float inv = 1.0f / (kLf ? 16.0f * kLevels * Lf : 16.0f * Lf);
         const float* sv = prm.sv + static_cast<size_t>(bh) * D;
         const float* Fsf = reinterpret_cast<const float*>(Fs);
         __nv_bfloat16* orow = prm.out + (static_cast<size_t>(bh) * prm.N + row) * D;
@@ -643,7 +677,8 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
           for (int u = 0; u < 4; ++u) dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
         }
-        if (prm.lse && hh == 0) prm.lse[static_cast<size_t>(bh) * prm.N + row] = m_ref + logf(Lf * (1.0f / 15.0f));
+        if (prm.lse && hh == 0)
+          prm.lse[static_cast<size_t>(bh) * prm.N + row] = m_ref + logf(kLf ? Lf : Lf * (1.0f / kLevels));
       }
     }
     if (!ok) set_status(kStatusTimeout);
@@ -682,7 +717,7 @@ bool make_code_map(CUtensorMap* m, const void* base, int BH, int N, int D, int r
   return r == CUDA_SUCCESS;
 }
 
-template <int D, int BN, bool DUMP>
+template <int D, int BN, bool DUMP, int MODE>
 cudaError_t launch_cfg(const ra_problem& p, const uint8_t* q4, const uint8_t* k4, const uint8_t* v4,
                        const AttnParams& prm, cudaStream_t st) {
   using C = Cfg<D, BN>;
@@ -691,7 +726,7 @@ cudaError_t launch_cfg(const ra_problem& p, const uint8_t* q4, const uint8_t* k4
   if (!make_code_map(&mq, q4, BH, p.N, D, kRows) || !make_code_map(&mk, k4, BH, p.N, D, BN) ||
       !make_code_map(&mv, v4, BH, p.N, D, BN))
     return cudaErrorInvalidValue;
-  auto kern = attn_int4_kernel<D, BN, DUMP>;
+  auto kern = attn_int4_kernel<D, BN, DUMP, MODE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
   int dev = 0, nsm = 0;
@@ -706,7 +741,7 @@ cudaError_t launch_cfg(const ra_problem& p, const uint8_t* q4, const uint8_t* k4
 
 cudaError_t launch_attn_int4(const ra_problem& p, const uint8_t* q4, const float* sq, const uint8_t* k4,
                              const float* sk, const uint8_t* v4, const float* sv, void* out, float* lse,
-                             const AttnDump* dump, cudaStream_t st, int* unsupported) {
+                             const AttnDump* dump, int mode, cudaStream_t st, int* unsupported) {
   AttnParams prm{};
   prm.N = p.N;
   prm.BH = p.B * p.H;
@@ -723,15 +758,27 @@ cudaError_t launch_attn_int4(const ra_problem& p, const uint8_t* q4, const float
     prm.dump_s = dump->s; prm.dump_p = dump->p; prm.dump_acc = dump->acc;
   }
   *unsupported = 0;
-#define RA_CASE(DD, BB)                                                                              \
-  if (p.D == DD && p.block_k == BB)                                                                  \
-    return dmp ? launch_cfg<DD, BB, true>(p, q4, k4, v4, prm, st) : launch_cfg<DD, BB, false>(p, q4, k4, v4, prm, st);
-  RA_CASE(128, 64)
-  RA_CASE(128, 32)
-  RA_CASE(128, 16)
-  RA_CASE(64, 64)
-  RA_CASE(64, 32)
-  RA_CASE(64, 16)
+#define RA_CASE(DD, BB, MM)                                                                          \
+  if (p.D == DD && p.block_k == BB && mode == MM)                                                    \
+    return dmp ? launch_cfg<DD, BB, true, MM>(p, q4, k4, v4, prm, st)                                \
+               : launch_cfg<DD, BB, false, MM>(p, q4, k4, v4, prm, st);
+  RA_CASE(128, 64, 0)
+  RA_CASE(128, 32, 0)
+  RA_CASE(128, 16, 0)
+  RA_CASE(64, 64, 0)
+  RA_CASE(64, 32, 0)
+  RA_CASE(64, 16, 0)
+  // Ablation modes: block_k = 64 only.
+  RA_CASE(128, 64, 1)
+  RA_CASE(128, 64, 2)
+  RA_CASE(128, 64, 4)
+  RA_CASE(128, 64, 5)
+  RA_CASE(128, 64, 6)
+  RA_CASE(64, 64, 1)
+  RA_CASE(64, 64, 2)
+  RA_CASE(64, 64, 4)
+  RA_CASE(64, 64, 5)
+  RA_CASE(64, 64, 6)
 #undef RA_CASE
   *unsupported = 1;
   return cudaSuccess;

@@ -71,16 +71,32 @@ ra_status ra_rope_rotate_quant(const ra_problem* p, int in_dtype, const void* q,
                                        workspace, static_cast<cudaStream_t>(stream)));
 }
 
+// Kernel mode bits from the ablation options (0 = the method's defaults).
+static bool attn_mode(const ra_attn_opts* o, int* mode) {
+  if (!o) { *mode = 0; return true; }
+  if (o->p_mode < RA_P_RANGE || o->p_mode > RA_P_SYMMETRIC || o->l_mode < RA_L_CODES || o->l_mode > RA_L_FP32)
+    return false;
+  *mode = o->p_mode | (o->l_mode == RA_L_FP32 ? 4 : 0);
+  return true;
+}
+
 ra_status ra_attn_int4(const ra_problem* p, const uint8_t* q4, const float* sq, const uint8_t* k4,
                        const float* sk, const uint8_t* v4, const float* sv, void* out, float* lse,
                        void* stream) {
-  if (!valid_problem(p)) return RA_ERR_INVALID_ARG;
+  return ra_attn_int4_opts(p, nullptr, q4, sq, k4, sk, v4, sv, out, lse, stream);
+}
+
+ra_status ra_attn_int4_opts(const ra_problem* p, const ra_attn_opts* opts, const uint8_t* q4, const float* sq,
+                            const uint8_t* k4, const float* sk, const uint8_t* v4, const float* sv, void* out,
+                            float* lse, void* stream) {
+  int mode = 0;
+  if (!valid_problem(p) || !attn_mode(opts, &mode)) return RA_ERR_INVALID_ARG;
   const void* ptrs[] = {q4, sq, k4, sk, v4, sv, out};
   for (const void* x : ptrs)
     if (!aligned16(x)) return RA_ERR_INVALID_ARG;
   if (!aligned16_or_null(lse)) return RA_ERR_INVALID_ARG;
   int unsupported = 0;
-  cudaError_t e = ra::launch_attn_int4(*p, q4, sq, k4, sk, v4, sv, out, lse, nullptr,
+  cudaError_t e = ra::launch_attn_int4(*p, q4, sq, k4, sk, v4, sv, out, lse, nullptr, mode,
                                        static_cast<cudaStream_t>(stream), &unsupported);
   if (unsupported) return RA_ERR_UNSUPPORTED;
   return from_cuda(e);
@@ -90,7 +106,16 @@ ra_status ra_test_int4_codes(const ra_problem* p, const uint8_t* q4, const float
                              const float* sk, const uint8_t* v4, const float* sv, int b, int h, int q_tile,
                              int32_t* s_dump, int8_t* p_dump, int32_t* acc_dump, void* out, float* lse,
                              void* stream) {
-  if (!valid_problem(p)) return RA_ERR_INVALID_ARG;
+  return ra_test_int4_codes_opts(p, nullptr, q4, sq, k4, sk, v4, sv, b, h, q_tile, s_dump, p_dump, acc_dump,
+                                 out, lse, stream);
+}
+
+ra_status ra_test_int4_codes_opts(const ra_problem* p, const ra_attn_opts* opts, const uint8_t* q4,
+                                  const float* sq, const uint8_t* k4, const float* sk, const uint8_t* v4,
+                                  const float* sv, int b, int h, int q_tile, int32_t* s_dump, int8_t* p_dump,
+                                  int32_t* acc_dump, void* out, float* lse, void* stream) {
+  int mode = 0;
+  if (!valid_problem(p) || !attn_mode(opts, &mode)) return RA_ERR_INVALID_ARG;
   const void* ptrs[] = {q4, sq, k4, sk, v4, sv, out};
   for (const void* x : ptrs)
     if (!aligned16(x)) return RA_ERR_INVALID_ARG;
@@ -106,7 +131,7 @@ ra_status ra_test_int4_codes(const ra_problem* p, const uint8_t* q4, const float
   d.p = p_dump;
   d.acc = acc_dump;
   int unsupported = 0;
-  cudaError_t e = ra::launch_attn_int4(*p, q4, sq, k4, sk, v4, sv, out, lse, &d,
+  cudaError_t e = ra::launch_attn_int4(*p, q4, sq, k4, sk, v4, sv, out, lse, &d, mode,
                                        static_cast<cudaStream_t>(stream), &unsupported);
   if (unsupported) return RA_ERR_UNSUPPORTED;
   return from_cuda(e);

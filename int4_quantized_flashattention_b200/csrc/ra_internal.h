@@ -36,7 +36,7 @@ struct AttnDump {
 };
 cudaError_t launch_attn_int4(const ra_problem& p, const uint8_t* q4, const float* sq, const uint8_t* k4,
                              const float* sk, const uint8_t* v4, const float* sv, void* out, float* lse,
-                             const AttnDump* dump, cudaStream_t st, int* unsupported);
+                             const AttnDump* dump, int mode, cudaStream_t st, int* unsupported);
 cudaError_t read_attn_int4_status(uint32_t* out);
 cudaError_t read_attn_int4_diag(uint32_t* out);  // first timed-out wait site (diagnosis)
 

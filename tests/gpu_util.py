@@ -29,13 +29,13 @@ def to_device(x, wl, dev):
     return t("q"), t("k"), t("v"), torch.from_numpy(x["pos"]).to(dev)
 
 
-def gpu_forward(ra, wl, x, dev, with_lse=False):
+def gpu_forward(ra, wl, x, dev, with_lse=False, p_mode=0, l_mode=0):
     import torch
     p = problem_for(ra, wl)
     q, k, v, pos = to_device(x, wl, dev)
     codes = ra.rope_rotate_quant(p, q, k, v, pos)
     lse = torch.empty(wl.B, wl.H, wl.N, dtype=torch.float32, device=dev) if with_lse else None
-    out = ra.attn_int4(p, codes, lse=lse)
+    out = ra.attn_int4(p, codes, lse=lse, p_mode=p_mode, l_mode=l_mode)
     assert ra.sync_status() == 0
     host = {k2: t.cpu().numpy() for k2, t in codes.items()}
     host["out"] = out.float().cpu().numpy()

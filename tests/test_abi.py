@@ -28,7 +28,8 @@ def ra():
 def test_header_declares_the_entry_points():
     names = _declared()
     for n in ("ra_rope_rotate_quant", "ra_attn_int4", "ra_attn_bf16_fallback", "ra_test_int4_codes",
-              "ra_rope_bf16", "ra_workspace_bytes", "ra_sync_status", "ra_status_string"):
+              "ra_rope_bf16", "ra_workspace_bytes", "ra_sync_status", "ra_status_string",
+              "ra_attn_int4_opts", "ra_test_int4_codes_opts"):
         assert n in names
 
 
@@ -108,6 +109,23 @@ def test_block_k_128_is_reported_unsupported(ra):
     p = _wan(ra, block_k=128)
     good = C.c_void_p(0x10000)
     assert ra.lib().ra_attn_int4(C.byref(p), *([good] * 7), None, None) == 2
+
+
+def test_ablation_options_are_validated_before_any_launch(ra):
+    """Out-of-range switches are invalid; switches other than the defaults are
+    implemented for block_k = 64 only."""
+    good = C.c_void_p(0x10000)
+    L = ra.lib()
+    p = _wan(ra)
+    for pm, lm in ((3, 0), (-1, 0), (0, 2)):
+        opts = ra.AttnOpts(pm, lm)
+        assert L.ra_attn_int4_opts(C.byref(p), C.byref(opts), *([good] * 7), None, None) == 1
+        assert L.ra_test_int4_codes_opts(C.byref(p), C.byref(opts), *([good] * 6), 0, 0, 0,
+                                         None, None, None, good, None, None) == 1
+    p32 = _wan(ra, block_k=32)
+    for pm, lm in ((1, 0), (2, 0), (0, 1)):
+        opts = ra.AttnOpts(pm, lm)
+        assert L.ra_attn_int4_opts(C.byref(p32), C.byref(opts), *([good] * 7), None, None) == 2
 
 
 def test_test_entry_rejects_bad_tile(ra):

@@ -60,15 +60,17 @@ def _check_prologue(orc, wl, x, host, heads):
 TIE_WINDOW = 2e-4
 
 
-def _running_max_scores(wl, hc, rows):
-    """fp32 S (reading R9) and the running block maximum M of the given rows."""
+def _running_max_scores(wl, hc, rows, local=False):
+    """fp32 S (reading R9) and the maximum M the codes are taken against: the
+    running block maximum, or each block's own maximum (local)."""
     q = orc_unpack(hc["q4"]).astype(np.int64)[rows]
     k = orc_unpack(hc["k4"]).astype(np.int64)
     ci = hc["sq"][rows].astype(np.float32) * np.float32(1.0 / np.sqrt(wl.D))
     S = ((q @ k.T).astype(np.float32) * hc["sk"][None, :].astype(np.float32)) * ci[:, None]
     Bk = wl.block_k
     nb = -(-wl.N // Bk)
-    run = np.maximum.accumulate(np.stack([S[:, t * Bk:(t + 1) * Bk].max(1) for t in range(nb)], 1), axis=1)
+    bmax = np.stack([S[:, t * Bk:(t + 1) * Bk].max(1) for t in range(nb)], 1)
+    run = bmax if local else np.maximum.accumulate(bmax, axis=1)
     return S, np.repeat(run, Bk, axis=1)[:, :wl.N]
 
 
@@ -81,9 +83,12 @@ class TileCheck:
     """Checks query tiles of one head through the test entry and accumulates the
     end-to-end error over every tile checked."""
 
-    def __init__(self, ra, orc, wl, p, codes, host):
+    def __init__(self, ra, orc, wl, p, codes, host, p_mode=0, l_mode=0):
         self.ra, self.orc, self.wl, self.p, self.codes, self.host = ra, orc, wl, p, codes, host
-        self.po = orc.problem(wl)
+        self.p_mode, self.l_mode = p_mode, l_mode
+        self.po = orc.problem(wl, p_mode=p_mode, l_mode=l_mode)
+        self.levels = 7.0 if p_mode == orc.P_SYMMETRIC else 15.0
+        self.zp = 0 if p_mode == orc.P_SYMMETRIC else 8
         self.num = 0.0
         self.den = 0.0
         self.flips = 0
@@ -93,7 +98,8 @@ class TileCheck:
         ra, orc, wl, host = self.ra, self.orc, self.wl, self.host
         r0, r1 = tile * 128, min(tile * 128 + 128, wl.N)
         R = r1 - r0
-        out, lse, s, pc, acc = ra.test_int4_codes(self.p, self.codes, 0, h, tile)
+        out, lse, s, pc, acc = ra.test_int4_codes(self.p, self.codes, 0, h, tile, p_mode=self.p_mode,
+                                                  l_mode=self.l_mode)
         assert ra.sync_status() == 0
         s, pc, acc = s.cpu().numpy()[:R], pc.cpu().numpy()[:R], acc.cpu().numpy()[:R]
         hc = gu.head_codes(host, (0, h))
@@ -105,12 +111,12 @@ class TileCheck:
         bad = np.nonzero(diff)
         if len(bad[0]):
             assert np.abs(diff).max() <= 1
-            S, M = _running_max_scores(wl, hc, np.arange(r0, r1))
-            e15 = 15.0 * np.exp(S[bad].astype(np.float64) - M[bad].astype(np.float64))
+            S, M = _running_max_scores(wl, hc, np.arange(r0, r1), local=self.p_mode == orc.P_LOCAL)
+            e15 = self.levels * np.exp(S[bad].astype(np.float64) - M[bad].astype(np.float64))
             tie = np.abs(e15 - (np.floor(e15) + 0.5))
             assert np.all(tie <= TIE_WINDOW), (h, tile, tie.max())
         self.flips += len(bad[0])
-        self.relevant += int((ref["codes"] > -8).sum())
+        self.relevant += int((ref["codes"] > -self.zp).sum())
         assert np.mean(diff == 0) >= CODE_EXACT
         # integer P.V accumulators bit-exact on the kernel's own codes
         v = orc_unpack(hc["v4"]).astype(np.int64)
@@ -118,8 +124,8 @@ class TileCheck:
         for t in range(-(-wl.N // Bk)):
             sl = slice(t * Bk, min((t + 1) * Bk, wl.N))
             c = pc[:, sl].astype(np.int64)
-            assert np.array_equal(acc[:, t], (c + 8) @ v[sl])
-            assert np.array_equal(acc[:, t], c @ v[sl] + 8 * hc["colsum"][t][None, :])
+            assert np.array_equal(acc[:, t], (c + self.zp) @ v[sl])
+            assert np.array_equal(acc[:, t], c @ v[sl] + self.zp * hc["colsum"][t][None, :])
         # O on the kernel's own codes: relative L2 <= 1e-3 per tile
         got = host["out"][0, h, r0:r1]
         assert np.all(np.isfinite(got))
@@ -266,3 +272,36 @@ def test_repeat_runs_are_bitwise_identical(ra, dev):
         out = ra.attn_int4(p, codes)
         assert ra.sync_status() == 0
         assert torch.equal(out.float(), first)
+
+
+@pytest.mark.parametrize("p_mode,l_mode", [(0, 1), (1, 0), (1, 1), (2, 0), (2, 1)])
+@pytest.mark.parametrize("name,shape", [
+    ("small", None),
+    ("small", dict(D=128, seg=(44, 42, 42), block_k=64, grid=(2, 10, 10), H=2)),   # N = 200, ragged
+    ("small", dict(D=64, seg=(24, 20, 20), block_k=64, grid=(5, 9, 11), H=2)),     # D = 64, N = 495
+])
+def test_ablation_switches(ra, dev, orc, p_mode, l_mode, name, shape):
+    """Block-local-max codes, symmetric codes and the fp32 denominator (the
+    alternatives of key design 2) against the oracle's switches: S_int and the
+    accumulators bit-exact, codes within the exponential's tie window, O within
+    1e-3 on the kernel's own codes and end to end."""
+    wl = si.WORKLOADS[name] if shape is None else si.WORKLOADS[name].with_(name=f"abl_{shape['D']}", **shape)
+    x = si.make_inputs(wl)
+    p, codes, host = gu.gpu_forward(ra, wl, x, dev, with_lse=True, p_mode=p_mode, l_mode=l_mode)
+    tc = TileCheck(ra, orc, wl, p, codes, host, p_mode=p_mode, l_mode=l_mode)
+    for h in range(wl.H):
+        tc.head(h)
+    assert tc.end_to_end() <= 1e-3
+
+
+def test_ablation_switches_change_the_result(ra, dev, orc):
+    """Each switch really changes the output (the modes are not silently equal)."""
+    wl = si.WORKLOADS["small"]
+    x = si.make_inputs(wl)
+    outs = {}
+    for pm, lm in ((0, 0), (0, 1), (1, 0), (2, 0)):
+        outs[(pm, lm)] = gu.gpu_forward(ra, wl, x, dev, p_mode=pm, l_mode=lm)[2]["out"]
+    base = outs[(0, 0)]
+    for key, o in outs.items():
+        if key != (0, 0):
+            assert gu.rel_l2(o, base) > 1e-3, key
