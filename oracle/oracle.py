@@ -91,6 +91,8 @@ def rope_tables(p: OrcProblem):
 
 def rope_rotate(p: OrcProblem, x: np.ndarray, pos: np.ndarray, swap_order: bool = False) -> np.ndarray:
     """RoPE + rotation of one head's rows x [N, D] (fp32), per the oracle's rules."""
+    if x.shape != (p.N, p.D) or len(pos) != p.N:
+        raise ValueError(f"rope_rotate: x {x.shape} / pos {len(pos)} do not match N={p.N}, D={p.D}")
     x = np.ascontiguousarray(x, np.float32)
     pos = np.ascontiguousarray(pos, np.int32)
     out = np.empty_like(x)

@@ -59,7 +59,7 @@ typedef struct {
   int seg[3];     /* frame / height / width channel counts, sum = D */
   int grid[3];    /* frame / height / width extents of the token grid */
   double theta;   /* RoPE base */
-  int rot;        /* 0 = RoPE only, 1 = interleaved rotation, 2 = half rotation */
+  int rot;        /* 0 = RoPE only, 1 = interleaved, 2 = half, 3 = full Hadamard rotation */
   int block_q, block_k;
   int p_mode;     /* ORC_P_RANGE (default), ORC_P_LOCAL, ORC_P_SYMMETRIC (R11) */
   int l_mode;     /* ORC_L_CODES (default), ORC_L_FP32 (R11) */
@@ -83,7 +83,8 @@ static int check_problem(const orc_problem* p) {
     if (p->grid[j] < 1) return ORC_BAD;
   }
   if (p->grid[0] * p->grid[1] * p->grid[2] < 1) return ORC_BAD;
-  if (p->rot < 0 || p->rot > 2 || p->block_k < 1) return ORC_BAD;
+  if (p->rot < 0 || p->rot > 3 || p->block_k < 1) return ORC_BAD;
+  if (p->rot == 3 && (p->D & (p->D - 1))) return ORC_BAD;  /* Sylvester H_D needs D = 2^k */
   if (p->p_mode < ORC_P_RANGE || p->p_mode > ORC_P_SYMMETRIC) return ORC_BAD;
   if (p->l_mode < ORC_L_CODES || p->l_mode > ORC_L_FP32) return ORC_BAD;
   return ORC_OK;
@@ -139,6 +140,11 @@ int orc_rope_tables(const orc_problem* p, float* tab_a, float* tab_b) {
  *                then per segment, h = Dj/2, i < h:
  *                out[2i] = (r_i + r_{i+h}) * (1/sqrt2), out[2i+1] = (r_i - r_{i+h}) * (1/sqrt2)
  *   none       : RoPE only.
+ *   full       : RoPE (as half), then the whole row times H_D / sqrt(D), H_D
+ *                the Sylvester Hadamard matrix (the full D x D rotation of the
+ *                pages' ablation): butterflies (a, b) -> (a + b, a - b) on
+ *                channel pairs d apart for d = 1, 2, 4, ..., D/2 in that
+ *                order, then one multiplication by fp32(1/sqrt(D)).
  * swap_order != 0 applies the half-rotation before RoPE instead (used only by a
  * test that shows the other order breaks QK^T invariance).
  */
@@ -184,6 +190,18 @@ static void rope_rotate_row(const orc_problem* p, const float* ta, const float* 
       for (int d = 0; d < dj; ++d) out[o + d] = tmp[o + d];
     }
     base += p->grid[j] * npair;
+  }
+  if (p->rot == 3) {
+    const int D = p->D;
+    for (int d = 1; d < D; d <<= 1)
+      for (int i = 0; i < D; ++i)
+        if (!(i & d)) {
+          float a = out[i], b = out[i + d];
+          out[i] = a + b;
+          out[i + d] = a - b;
+        }
+    const float c = (float)(1.0 / sqrt((double)D));
+    for (int i = 0; i < D; ++i) out[i] = out[i] * c;
   }
 }
 
@@ -529,7 +547,8 @@ int orc_attention_exact_blocked_rows(const orc_problem* p, const double* q, cons
  *   interleaved: block-diagonal of D/2 copies of H2 on channel pairs (2i, 2i+1);
  *   half: per segment, a permutation placing channel i and i + Dj/2 at 2i, 2i+1,
  *         followed by Dj/2 copies of H2 on those adjacent pairs;
- *   none: the identity.
+ *   none: the identity;
+ *   full: the normalised Sylvester Hadamard matrix H_D / sqrt(D).
  */
 int orc_rotation_matrix(const orc_problem* p, double* R) {
   if (check_problem(p)) return ORC_BAD;
@@ -538,6 +557,15 @@ int orc_rotation_matrix(const orc_problem* p, double* R) {
   memset(R, 0, sizeof(double) * D * D);
   if (p->rot == 0) {
     for (int d = 0; d < D; ++d) R[d * D + d] = 1.0;
+    return ORC_OK;
+  }
+  if (p->rot == 3) {  /* H_D / sqrt(D), H_D[i][j] = (-1)^popcount(i & j) */
+    for (int i = 0; i < D; ++i)
+      for (int j = 0; j < D; ++j) {
+        int b = i & j, par = 0;
+        while (b) { par ^= b & 1; b >>= 1; }
+        R[i * D + j] = (par ? -1.0 : 1.0) / sqrt((double)D);
+      }
     return ORC_OK;
   }
   double* Pi = (double*)calloc((size_t)D * D, sizeof(double));

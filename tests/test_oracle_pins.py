@@ -34,7 +34,7 @@ def _prob(orc, rot, sp, **kw):
 
 # --- rotation: orthogonality and QK^T equivalence (key design 1: R must be in O(D)) ---
 
-@pytest.mark.parametrize("rot", [1, 2])
+@pytest.mark.parametrize("rot", [1, 2, 3])
 @pytest.mark.parametrize("sp", SPLITS)
 def test_rotation_is_orthogonal(orc, rot, sp):
     R = orc.rotation_matrix(_prob(orc, rot, sp))
@@ -42,7 +42,7 @@ def test_rotation_is_orthogonal(orc, rot, sp):
     assert err <= 1e-15
 
 
-@pytest.mark.parametrize("rot", [1, 2])
+@pytest.mark.parametrize("rot", [1, 2, 3])
 @pytest.mark.parametrize("sp", SPLITS)
 def test_rotation_preserves_qk(orc, rot, sp):
     rng = np.random.default_rng(7)
@@ -147,7 +147,7 @@ def test_fused_interleaved_stays_block_diagonal(orc, rot):
         assert np.any(Mp[~mask] != 0.0)
 
 
-@pytest.mark.parametrize("rot", [0, 1, 2])
+@pytest.mark.parametrize("rot", [0, 1, 2, 3])
 @pytest.mark.parametrize("sp", SPLITS)
 def test_elementwise_prologue_equals_matrix_form(orc, rot, sp):
     """The fp32 elementwise RoPE+rotation equals x M_n R in fp64 up to fp32 rounding."""
@@ -532,3 +532,59 @@ def test_fp32_l_changes_only_the_denominator(orc):
         ratio = np.exp(a["lse"] - b["lse"])          # l_codes / l_fp32
         assert np.abs(b["out"] - a["out"] * ratio[:, None]).max() <= 1e-12 * np.abs(a["out"]).max()
         assert np.all(ratio > 0) and not np.allclose(ratio, 1.0)
+
+
+# --- full D x D Hadamard rotation (the pages' ablation; a third rotation mode) ---
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_full_rotation_is_the_normalised_sylvester_hadamard(orc, D):
+    """The oracle's matrix equals scipy's Sylvester Hadamard matrix / sqrt(D)."""
+    from scipy.linalg import hadamard
+    sp = SPLITS[0] if D == 64 else SPLITS[1]
+    R = orc.rotation_matrix(_prob(orc, 3, sp))
+    assert np.array_equal(R, hadamard(D).astype(np.float64) / math.sqrt(D))
+
+
+def test_full_rotation_mixes_every_channel(orc):
+    """Unlike the 2x2 rotations, every output channel depends on every input."""
+    sp = SPLITS[1]
+    p = _prob(orc, 3, sp, N=1)
+    pos = si.positions(sp["grid"])[:1]
+    for d in (0, 63, 127):
+        x = np.zeros((1, sp["D"]), np.float32)
+        x[0, d] = 1.0
+        y = orc.rope_rotate(p, x, pos)   # position (0, 0, 0): RoPE is the identity
+        assert np.all(np.abs(np.abs(y) - 1 / math.sqrt(sp["D"])) <= 1e-7)
+
+
+def test_full_rotation_butterflies_follow_the_stated_order(orc):
+    """fp32 transform equals the same butterfly sequence written out in numpy
+    float32 (stage distances 1, 2, ..., D/2, then one scaling)."""
+    sp = SPLITS[1]
+    p = _prob(orc, 3, sp, N=1)
+    pos = si.positions(sp["grid"])[:1]
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((1, sp["D"])).astype(np.float32) * np.float32(20)
+    y = orc.rope_rotate(p, x, pos)[0]
+    z = x[0].copy()
+    d = 1
+    while d < sp["D"]:
+        idx = np.array([i for i in range(sp["D"]) if not i & d])
+        a, b = z[idx].copy(), z[idx + d].copy()
+        z[idx], z[idx + d] = a + b, a - b
+        d *= 2
+    z = z * np.float32(1 / math.sqrt(sp["D"]))
+    assert np.array_equal(y, z)
+
+
+def test_full_rotation_flattens_outlier_channels(orc):
+    """Hadamard spreads the outlier channels over all channels: the per-token
+    amax relative to the RMS falls (what makes INT4 codes finer)."""
+    wl = si.WORKLOADS["small"]
+    x = si.make_inputs(wl, heads=(0,))
+    ratio = {}
+    for rot in (0, 3):
+        p = orc.problem(wl.with_(rot=rot))
+        y = orc.rope_rotate(p, x["q"][0, 0], x["pos"]).astype(np.float64)
+        ratio[rot] = np.mean(np.abs(y).max(1) / np.sqrt((y ** 2).mean(1)))
+    assert ratio[3] < 0.6 * ratio[0]
