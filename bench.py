@@ -308,6 +308,29 @@ def run_ours(args, rank, world, local_rank):
                 raise RuntimeError(f"device status not ok after the {name} ablation")
             abl[name] = statistics.median(ts)
 
+    # The prologue under each rotation mode (full D x D Hadamard against the
+    # 2x2 rotations), timed on the same inputs after everything else.
+    rot_ms = {}
+    for rname, rmode in (("interleaved", ra.ROT_INTERLEAVED), ("half", ra.ROT_HALF), ("full", ra.ROT_FULL),
+                         ("none", ra.ROT_NONE)):
+        pr = ra.Problem.make(wl.B, wl.H, wl.D, wl.seg, wl.grid, theta=wl.theta, rot=rmode,
+                             block_q=wl.block_q, block_k=wl.block_k)
+        for _ in range(2):
+            ra.rope_rotate_quant(pr, q, k, v, pos, out=codes, workspace=ws)
+        torch.cuda.synchronize(dev)
+        ts = []
+        for _ in range(max(3, args.steps // 4)):
+            a0 = torch.cuda.Event(enable_timing=True)
+            a1 = torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            ra.rope_rotate_quant(pr, q, k, v, pos, out=codes, workspace=ws)
+            a1.record(stream)
+            torch.cuda.synchronize(dev)
+            ts.append(a0.elapsed_time(a1))
+        if ra.sync_status() != 0:
+            raise RuntimeError(f"device status not ok after the {rname} prologue")
+        rot_ms[rname] = statistics.median(ts)
+
     ops = wl.attn_ops()
     ms_step = total_ms / args.steps
     value = weak_scaling_value(world, ops, ms_step)
@@ -338,6 +361,7 @@ def run_ours(args, rank, world, local_rank):
                           "kernel": "attn_bf16_kernel", "note": "4N^2DH flops of bf16 attention on the RoPE'd inputs"},
         "ablations": {n: {"ms": round(t, 4), "tops": round(ops / (t * 1e-3) / 1e12, 1),
                           "frac": round(ops / (t * 1e-3) / 1e12 / int8_peak, 4)} for n, t in abl.items()},
+        "prologue_by_rotation_ms": {n: round(t, 4) for n, t in rot_ms.items()},
         "gpu_launches": KERNELS_PER_STEP * args.steps,
         "clocks": clk.summary(),
     }

@@ -51,7 +51,10 @@ typedef enum {
 typedef enum {
   RA_ROT_NONE = 0,         /* 3D RoPE only */
   RA_ROT_INTERLEAVED = 1,  /* H2 blocks on adjacent channel pairs, fused into the RoPE tables */
-  RA_ROT_HALF = 2          /* per segment: pair channel i with i + Dj/2, then H2 blocks */
+  RA_ROT_HALF = 2,         /* per segment: pair channel i with i + Dj/2, then H2 blocks */
+  RA_ROT_FULL = 3          /* the whole row times H_D / sqrt(D) (Sylvester Hadamard), after
+                              RoPE: the pages' full-rotation ablation (papernotes page,
+                              ablation on rotation granularity) */
 } ra_rot_mode;
 
 typedef enum { RA_DT_F32 = 0, RA_DT_BF16 = 1 } ra_dtype;

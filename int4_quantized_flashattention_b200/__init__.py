@@ -15,12 +15,12 @@ from typing import Dict, Optional, Sequence
 import torch
 
 __all__ = [
-    "ROT_NONE", "ROT_INTERLEAVED", "ROT_HALF", "RaError", "Problem", "lib", "workspace_bytes",
+    "ROT_NONE", "ROT_INTERLEAVED", "ROT_HALF", "ROT_FULL", "RaError", "Problem", "lib", "workspace_bytes",
     "rope_rotate_quant", "attn_int4", "test_int4_codes", "rope_bf16", "attn_bf16_fallback",
     "sync_status", "library_path", "AttnOpts", "P_RANGE", "P_LOCAL_MAX", "P_SYMMETRIC", "L_CODES", "L_FP32",
 ]
 
-ROT_NONE, ROT_INTERLEAVED, ROT_HALF = 0, 1, 2
+ROT_NONE, ROT_INTERLEAVED, ROT_HALF, ROT_FULL = 0, 1, 2, 3
 DT_F32, DT_BF16 = 0, 1
 P_RANGE, P_LOCAL_MAX, P_SYMMETRIC = 0, 1, 2   # ra_attn_opts.p_mode
 L_CODES, L_FP32 = 0, 1                        # ra_attn_opts.l_mode

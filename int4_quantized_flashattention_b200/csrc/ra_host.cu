@@ -29,7 +29,7 @@ bool valid_problem(const ra_problem* p) {
   }
   if (sum != p->D) return false;
   if (!(p->theta > 0.0f) || !std::isfinite(p->theta)) return false;
-  if (p->rot < RA_ROT_NONE || p->rot > RA_ROT_HALF) return false;
+  if (p->rot < RA_ROT_NONE || p->rot > RA_ROT_FULL) return false;
   const int bq = p->block_q, bk = p->block_k;
   if (bq != 16 && bq != 32 && bq != 64 && bq != 128) return false;
   if (bk != 16 && bk != 32 && bk != 64 && bk != 128) return false;

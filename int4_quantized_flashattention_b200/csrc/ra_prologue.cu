@@ -32,6 +32,8 @@ struct SegInfo {
   int dj[3];      // channels of each segment
   int toff[3];    // first table entry of each segment
   int grid[3];
+  int D;
+  float hscale;   // fp32 rounding of 1/sqrt(D), the full rotation's scale
 };
 
 __device__ __forceinline__ void load8(const void* base, size_t elem_off, int dtype, float* x) {
@@ -182,7 +184,36 @@ __device__ __forceinline__ void rope_coef8p(const SegInfo& s, const RopePlan& rp
   }
 }
 
-// The same arithmetic as rope_rotate8, from coefficients already loaded.
+// Full rotation: the token row times H_D / sqrt(D) (Sylvester Hadamard), as
+// butterflies (a, b) -> (a + b, a - b) on channels d apart, d = 1, 2, ..., D/2
+// in that order, then one fp32 scaling.  The thread holds channels
+// [c0, c0 + 8): distances 1, 2, 4 are in its registers, distances 8 ... D/2
+// pair it with the lanes 1 ... D/16 apart in its token's lane group.
+__device__ __forceinline__ void hadamard8(const SegInfo& s, int c0, float* x) {
+#pragma unroll
+  for (int d = 1; d < 8; d <<= 1)
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if (!(i & d)) {
+        const float a = x[i], b = x[i + d];
+        x[i] = __fadd_rn(a, b);
+        x[i + d] = __fsub_rn(a, b);
+      }
+  const int g = c0 >> 3;  // this thread's place among the token's D/8 lanes
+  for (int m = 1; m < (s.D >> 3); m <<= 1) {
+    const bool upper = (g & m) != 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float o = __shfl_xor_sync(0xFFFFFFFFu, x[i], m);
+      x[i] = upper ? __fsub_rn(o, x[i]) : __fadd_rn(x[i], o);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) x[i] = __fmul_rn(x[i], s.hscale);
+}
+
+// The same arithmetic as rope_rotate8, from coefficients already loaded (rot
+// 3: the full Hadamard rotation after the RoPE pairs).
 __device__ __forceinline__ void rope_apply8(const SegInfo& s, int rot, const float* ca, const float* cb, int c0,
                                             float* x, float* row) {
 #pragma unroll
@@ -213,6 +244,7 @@ __device__ __forceinline__ void rope_apply8(const SegInfo& s, int rot, const flo
     }
     __syncwarp();
   }
+  if (rot == 3) hadamard8(s, c0, x);
 }
 
 
@@ -599,6 +631,8 @@ SegInfo seg_info(const ra_problem& p) {
     o += p.seg[j];
     t += p.grid[j] * (p.seg[j] / 2);
   }
+  s.D = p.D;
+  s.hscale = static_cast<float>(1.0 / sqrt(static_cast<double>(p.D)));
   return s;
 }
 

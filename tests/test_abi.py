@@ -64,7 +64,7 @@ def test_workspace_bytes(ra):
 
 
 @pytest.mark.parametrize("field,value", [
-    ("D", 96), ("N", 0), ("block_k", 48), ("block_q", 100), ("rot", 3), ("theta", -1.0), ("B", 0),
+    ("D", 96), ("N", 0), ("block_k", 48), ("block_q", 100), ("rot", 4), ("theta", -1.0), ("B", 0),
 ])
 def test_invalid_problem_rejected(ra, field, value):
     p = _wan(ra)

@@ -171,6 +171,9 @@ def test_small_workloads_end_to_end(ra, dev, orc, name):
     (64, (24, 20, 20), 64, 1, (5, 9, 11)),      # N = 495, D = 64
     (64, (24, 20, 20), 32, 0, (1, 1, 7)),       # N = 7, no rotation
     (128, (44, 42, 42), 64, 2, (1, 1, 1)),      # N = 1
+    (128, (44, 42, 42), 64, 3, (2, 10, 10)),    # full Hadamard rotation, N = 200
+    (128, (16, 56, 56), 16, 3, (2, 5, 9)),      # full rotation, N = 90, block_k 16
+    (64, (24, 20, 20), 32, 3, (5, 9, 11)),      # full rotation, D = 64
 ])
 def test_shapes_and_ragged_tails(ra, dev, orc, D, seg, bk, rot, grid):
     wl = si.WORKLOADS["small"].with_(name=f"case{D}_{bk}", D=D, seg=seg, block_k=bk, rot=rot, grid=grid, H=3)
