@@ -149,6 +149,10 @@ __device__ __forceinline__ void unpack8(const Raw8<kBf16>& r, float* x) {
 // each of the thread's 4 channel pairs, computed once.
 struct RopePlan {
   int seg[4], off[4], stride[4];
+  // Half rotation: output channel c0 + i reads channels u and w = u + Dj/2 of
+  // the RoPE'd row and takes their sum (even) or difference (odd):
+  // hx[i] = u | w << 8 | odd << 16.
+  uint32_t hx[8];
   __device__ __forceinline__ void init(const SegInfo& s, int c0) {
 #pragma unroll
     for (int pr = 0; pr < 4; ++pr) {
@@ -157,6 +161,13 @@ struct RopePlan {
       seg[pr] = j;
       off[pr] = s.toff[j] + ((d - s.off[j]) >> 1);
       stride[pr] = s.dj[j] >> 1;
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int d = c0 + i;
+      const int j = seg_of(s, d);
+      const uint32_t u = static_cast<uint32_t>(s.off[j] + ((d - s.off[j]) >> 1));
+      hx[i] = u | ((u + (s.dj[j] >> 1)) << 8) | (static_cast<uint32_t>((d - s.off[j]) & 1) << 16);
     }
   }
 };
@@ -214,8 +225,8 @@ __device__ __forceinline__ void hadamard8(const SegInfo& s, int c0, float* x) {
 
 // The same arithmetic as rope_rotate8, from coefficients already loaded (rot
 // 3: the full Hadamard rotation after the RoPE pairs).
-__device__ __forceinline__ void rope_apply8(const SegInfo& s, int rot, const float* ca, const float* cb, int c0,
-                                            float* x, float* row) {
+__device__ __forceinline__ void rope_apply8(const SegInfo& s, const RopePlan& rp, int rot, const float* ca,
+                                            const float* cb, int c0, float* x, float* row) {
 #pragma unroll
   for (int pr = 0; pr < 4; ++pr) {
     const float a = ca[pr], b = cb[pr];
@@ -235,12 +246,9 @@ __device__ __forceinline__ void rope_apply8(const SegInfo& s, int rot, const flo
     __syncwarp();
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const int d = c0 + i;
-      const int j = seg_of(s, d);
-      const int h = s.dj[j] >> 1;
-      const int t = (d - s.off[j]) >> 1;
-      const float u = row[s.off[j] + t], w = row[s.off[j] + t + h];
-      x[i] = (d - s.off[j]) & 1 ? __fmul_rn(__fsub_rn(u, w), r2) : __fmul_rn(__fadd_rn(u, w), r2);
+      const uint32_t h = rp.hx[i];
+      const float u = row[h & 0xFFu], w = row[(h >> 8) & 0xFFu];
+      x[i] = (h >> 16) ? __fmul_rn(__fsub_rn(u, w), r2) : __fmul_rn(__fadd_rn(u, w), r2);
     }
     __syncwarp();
   }
@@ -348,8 +356,9 @@ __device__ __forceinline__ bool stage_wait(uint64_t* bar, uint32_t parity, volat
 }
 
 // Pass 1: per chunk of tokens, fp64 channel sums of the rotated K and channel
-// maxima of |V|.
-template <bool kBf16>
+// maxima of |V|.  kRot: the rotation mode (a template parameter, so every
+// mode keeps only its own per-thread state).
+template <bool kBf16, int kRot>
 __global__ void __launch_bounds__(kThreads, 3) prologue_reduce_kernel(PrologueArgs a) {
   using IO = StageIO<kBf16, 2>;
   __shared__ float rows[kThreads / 32][4][128];
@@ -401,7 +410,7 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_reduce_kernel(PrologueAr
       }
       // Every lane takes part (the half rotation synchronises the warp).
       rope_coef8p(a.s, rp, a.tab_a, a.tab_b, gp, ca, cb);
-      rope_apply8(a.s, a.rot, ca, cb, c0, x, rows[warp][tok_in_warp]);
+      rope_apply8(a.s, rp, kRot, ca, cb, c0, x, rows[warp][tok_in_warp]);
       if (valid) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -460,7 +469,7 @@ __global__ void prologue_finalize_kernel(PrologueArgs a) {
 // the RoPE coefficients; column sums are kept per thread while a warp stays in
 // one key block, then combined across the warp's tokens and added to shared
 // memory.
-template <bool kBf16>
+template <bool kBf16, int kRot>
 __global__ void __launch_bounds__(kThreads, 3) prologue_quant_kernel(PrologueArgs a) {
   using IO = StageIO<kBf16, 3>;
   __shared__ float rows[kThreads / 32][4][128];
@@ -540,8 +549,8 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_quant_kernel(PrologueArg
         for (int i = 0; i < 8; ++i) { xq[i] = 0.0f; xk[i] = 0.0f; xv[i] = 0.0f; }
       }
       rope_coef8p(a.s, rp, a.tab_a, a.tab_b, gp, ca, cb);
-      rope_apply8(a.s, a.rot, ca, cb, c0, xq, rows[warp][tok_in_warp]);
-      rope_apply8(a.s, a.rot, ca, cb, c0, xk, rows[warp][tok_in_warp]);
+      rope_apply8(a.s, rp, kRot, ca, cb, c0, xq, rows[warp][tok_in_warp]);
+      rope_apply8(a.s, rp, kRot, ca, cb, c0, xk, rows[warp][tok_in_warp]);
       float mq = 0.0f, mk = 0.0f;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -673,6 +682,22 @@ static cudaError_t launch_tables(const ra_problem& p, int rot, float* ta, float*
   return cudaGetLastError();
 }
 
+// The three passes (channel reduce, finalize, quantise) for one input type and
+// rotation mode.
+template <bool kBf16, int kRot>
+static cudaError_t launch_passes(const PrologueArgs& a, dim3 grid, int red_bytes, int quant_bytes,
+                                 cudaStream_t st) {
+  cudaError_t e;
+  if ((e = set_smem(prologue_reduce_kernel<kBf16, kRot>, red_bytes)) != cudaSuccess) return e;
+  prologue_reduce_kernel<kBf16, kRot><<<grid, kThreads, red_bytes, st>>>(a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  prologue_finalize_kernel<<<grid.y, 128, 0, st>>>(a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = set_smem(prologue_quant_kernel<kBf16, kRot>, quant_bytes)) != cudaSuccess) return e;
+  prologue_quant_kernel<kBf16, kRot><<<grid, kThreads, quant_bytes, st>>>(a);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_prologue(const ra_problem& p, int dtype, const void* q, const void* k, const void* v,
                             const int32_t* pos, uint8_t* q4, float* sq, uint8_t* k4, float* sk,
                             float* k_mean, uint8_t* v4, float* sv, int32_t* colsum, void* ws,
@@ -699,24 +724,18 @@ cudaError_t launch_prologue(const ra_problem& p, int dtype, const void* q, const
   const int el = dtype == 1 ? 2 : 4;
   const int red_bytes = kStg * 2 * kSub * p.D * el > kThreads * 8 * 12 ? kStg * 2 * kSub * p.D * el : kThreads * 8 * 12;
   const int quant_bytes = kStg * 3 * kSub * p.D * el;
-  if (dtype == 1) {
-    if ((e = set_smem(prologue_reduce_kernel<true>, red_bytes)) != cudaSuccess) return e;
-    prologue_reduce_kernel<true><<<grid, kThreads, red_bytes, st>>>(a);
-  } else {
-    if ((e = set_smem(prologue_reduce_kernel<false>, red_bytes)) != cudaSuccess) return e;
-    prologue_reduce_kernel<false><<<grid, kThreads, red_bytes, st>>>(a);
+  switch (dtype * 4 + p.rot) {
+#define RA_PRO(DT, ROT)                                                                              \
+  case DT * 4 + ROT:                                                                                 \
+    e = launch_passes<DT == 1, ROT>(a, grid, red_bytes, quant_bytes, st);                            \
+    break;
+    RA_PRO(0, 0) RA_PRO(0, 1) RA_PRO(0, 2) RA_PRO(0, 3)
+    RA_PRO(1, 0) RA_PRO(1, 1) RA_PRO(1, 2) RA_PRO(1, 3)
+#undef RA_PRO
+    default:
+      return cudaErrorInvalidValue;
   }
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  prologue_finalize_kernel<<<p.B * p.H, 128, 0, st>>>(a);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if (dtype == 1) {
-    if ((e = set_smem(prologue_quant_kernel<true>, quant_bytes)) != cudaSuccess) return e;
-    prologue_quant_kernel<true><<<grid, kThreads, quant_bytes, st>>>(a);
-  } else {
-    if ((e = set_smem(prologue_quant_kernel<false>, quant_bytes)) != cudaSuccess) return e;
-    prologue_quant_kernel<false><<<grid, kThreads, quant_bytes, st>>>(a);
-  }
-  return cudaGetLastError();
+  return e;
 }
 
 cudaError_t launch_rope_bf16(const ra_problem& p, int dtype, const void* q, const void* k,
