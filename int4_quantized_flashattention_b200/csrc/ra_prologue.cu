@@ -358,7 +358,7 @@ __device__ __forceinline__ bool stage_wait(uint64_t* bar, uint32_t parity, volat
 // Pass 1: per chunk of tokens, fp64 channel sums of the rotated K and channel
 // maxima of |V|.  kRot: the rotation mode (a template parameter, so every
 // mode keeps only its own per-thread state).
-template <bool kBf16, int kRot>
+template <bool kBf16, int kRot, int kD>
 __global__ void __launch_bounds__(kThreads, 3) prologue_reduce_kernel(PrologueArgs a) {
   using IO = StageIO<kBf16, 2>;
   __shared__ float rows[kThreads / 32][4][128];
@@ -366,12 +366,12 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_reduce_kernel(PrologueAr
   __shared__ int abort_flag;
   extern __shared__ __align__(128) uint8_t stg[];
   const int bh = blockIdx.y, chunk = blockIdx.x;
-  const int lpt = a.D >> 3, tpw = 32 / lpt;
+  const int lpt = kD >> 3, tpw = 32 / lpt;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tok_in_warp = lane / lpt, c0 = (lane % lpt) * 8;
   const int step = (kThreads / 32) * tpw;
   const int n0 = chunk * kChunk;
-  const size_t head = static_cast<size_t>(bh) * a.N * a.D;
+  const size_t head = static_cast<size_t>(bh) * a.N * kD;
   const void* src[2] = {a.k, a.v};
   RopePlan rp;
   rp.init(a.s, c0);
@@ -382,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_reduce_kernel(PrologueAr
   }
   __syncthreads();
   if (threadIdx.x == 0)
-    for (int sc = 0; sc < kStg; ++sc) IO::issue(src, head, a.D, a.N, n0, sc, stg, full);
+    for (int sc = 0; sc < kStg; ++sc) IO::issue(src, head, kD, a.N, n0, sc, stg, full);
   double ks[8];
   float vm[8];
 #pragma unroll
@@ -398,8 +398,8 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_reduce_kernel(PrologueAr
       int gp[3] = {0, 0, 0};
       if (valid) {
         Raw8<kBf16> rk, rv;
-        IO::read(stg, a.D, s, 0, ti, c0, rk);
-        IO::read(stg, a.D, s, 1, ti, c0, rv);
+        IO::read(stg, kD, s, 0, ti, c0, rk);
+        IO::read(stg, kD, s, 1, ti, c0, rv);
         unpack8<kBf16>(rk, x);
         unpack8<kBf16>(rv, y);
 #pragma unroll
@@ -420,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_reduce_kernel(PrologueAr
       }
     }
     __syncthreads();  // stage s consumed
-    if (threadIdx.x == 0 && sc + kStg < kChunk / kSub) IO::issue(src, head, a.D, a.N, n0, sc + kStg, stg, full);
+    if (threadIdx.x == 0 && sc + kStg < kChunk / kSub) IO::issue(src, head, kD, a.N, n0, sc + kStg, stg, full);
   }
   if (!ok) {
     if (threadIdx.x == 0) atomicOr(&g_prologue_status, kStatusTimeout);
@@ -433,7 +433,7 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_reduce_kernel(PrologueAr
 #pragma unroll
   for (int i = 0; i < 8; ++i) { red_s[threadIdx.x * 8 + i] = ks[i]; red_m[threadIdx.x * 8 + i] = vm[i]; }
   __syncthreads();
-  for (int d = threadIdx.x; d < a.D; d += kThreads) {
+  for (int d = threadIdx.x; d < kD; d += kThreads) {
     const int c = d >> 3, i = d & 7;
     double sum = 0.0;
     float mx = 0.0f;
@@ -441,7 +441,7 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_reduce_kernel(PrologueAr
       sum += red_s[t * 8 + i];
       mx = fmaxf(mx, red_m[t * 8 + i]);
     }
-    const size_t o = (static_cast<size_t>(bh) * a.nchunk + chunk) * a.D + d;
+    const size_t o = (static_cast<size_t>(bh) * a.nchunk + chunk) * kD + d;
     a.ksum[o] = sum;
     a.vmax[o] = mx;
   }
@@ -469,7 +469,7 @@ __global__ void prologue_finalize_kernel(PrologueArgs a) {
 // the RoPE coefficients; column sums are kept per thread while a warp stays in
 // one key block, then combined across the warp's tokens and added to shared
 // memory.
-template <bool kBf16, int kRot>
+template <bool kBf16, int kRot, int kD>
 __global__ void __launch_bounds__(kThreads, 3) prologue_quant_kernel(PrologueArgs a) {
   using IO = StageIO<kBf16, 3>;
   __shared__ float rows[kThreads / 32][4][128];
@@ -478,18 +478,18 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_quant_kernel(PrologueArg
   __shared__ int abort_flag;
   extern __shared__ __align__(128) uint8_t stg[];
   const int bh = blockIdx.y, chunk = blockIdx.x;
-  const int lpt = a.D >> 3, tpw = 32 / lpt;
+  const int lpt = kD >> 3, tpw = 32 / lpt;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tok_in_warp = lane / lpt, c0 = (lane % lpt) * 8;
   const int step = (kThreads / 32) * tpw;
   const int nblk = kChunk / a.block_k;
   const int n0 = chunk * kChunk;
-  const size_t head = static_cast<size_t>(bh) * a.N * a.D;
-  const size_t head4 = static_cast<size_t>(bh) * a.N * (a.D / 2);
+  const size_t head = static_cast<size_t>(bh) * a.N * kD;
+  const size_t head4 = static_cast<size_t>(bh) * a.N * (kD / 2);
   const void* src[3] = {a.q, a.k, a.v};
   RopePlan rp;
   rp.init(a.s, c0);
-  for (int i = threadIdx.x; i < nblk * a.D; i += kThreads) csum[i / a.D][i % a.D] = 0;
+  for (int i = threadIdx.x; i < nblk * kD; i += kThreads) csum[i / kD][i % kD] = 0;
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStg; ++s) mbar_init(full + s, 1);
     abort_flag = 0;
@@ -498,12 +498,12 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_quant_kernel(PrologueArg
   float kmean[8], vinv[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    kmean[i] = a.k_mean[bh * a.D + c0 + i];
-    vinv[i] = a.vinv[bh * a.D + c0 + i];
+    kmean[i] = a.k_mean[bh * kD + c0 + i];
+    vinv[i] = a.vinv[bh * kD + c0 + i];
   }
   __syncthreads();
   if (threadIdx.x == 0)
-    for (int sc = 0; sc < kStg; ++sc) IO::issue(src, head, a.D, a.N, n0, sc, stg, full);
+    for (int sc = 0; sc < kStg; ++sc) IO::issue(src, head, kD, a.N, n0, sc, stg, full);
   int cacc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   int cblk = (warp * tpw) / a.block_k;  // key block of this warp's first tokens
   // Adds this warp's per-thread column sums of block cblk to shared memory:
@@ -536,9 +536,9 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_quant_kernel(PrologueArg
       int gp[3] = {0, 0, 0};
       if (valid) {
         Raw8<kBf16> rq, rk, rv;
-        IO::read(stg, a.D, s, 0, ti, c0, rq);
-        IO::read(stg, a.D, s, 1, ti, c0, rk);
-        IO::read(stg, a.D, s, 2, ti, c0, rv);
+        IO::read(stg, kD, s, 0, ti, c0, rq);
+        IO::read(stg, kD, s, 1, ti, c0, rk);
+        IO::read(stg, kD, s, 2, ti, c0, rv);
         unpack8<kBf16>(rq, xq);
         unpack8<kBf16>(rk, xk);
         unpack8<kBf16>(rv, xv);
@@ -570,7 +570,7 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_quant_kernel(PrologueArg
         bv[i] = quant4_bits(xv[i], vinv[i]);
       }
       if (valid) {
-        const size_t o4 = head4 + static_cast<size_t>(n) * (a.D / 2) + (c0 >> 1);
+        const size_t o4 = head4 + static_cast<size_t>(n) * (kD / 2) + (c0 >> 1);
         *reinterpret_cast<uint32_t*>(a.q4 + o4) = pack8_bits(bq);
         *reinterpret_cast<uint32_t*>(a.k4 + o4) = pack8_bits(bk);
         *reinterpret_cast<uint32_t*>(a.v4 + o4) = pack8_bits(bv);
@@ -583,7 +583,7 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_quant_kernel(PrologueArg
       }
     }
     __syncthreads();  // stage s consumed
-    if (threadIdx.x == 0 && sc + kStg < kChunk / kSub) IO::issue(src, head, a.D, a.N, n0, sc + kStg, stg, full);
+    if (threadIdx.x == 0 && sc + kStg < kChunk / kSub) IO::issue(src, head, kD, a.N, n0, sc + kStg, stg, full);
   }
   if (!ok) {
     if (threadIdx.x == 0) atomicOr(&g_prologue_status, kStatusTimeout);
@@ -592,10 +592,10 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_quant_kernel(PrologueArg
   flush();
   __syncthreads();
   const int nb_total = (a.N + a.block_k - 1) / a.block_k;
-  for (int i = threadIdx.x; i < nblk * a.D; i += kThreads) {
-    const int bl = i / a.D, d = i % a.D;
+  for (int i = threadIdx.x; i < nblk * kD; i += kThreads) {
+    const int bl = i / kD, d = i % kD;
     const int gb = chunk * nblk + bl;
-    if (gb < nb_total) a.colsum[(static_cast<size_t>(bh) * nb_total + gb) * a.D + d] = csum[bl][d];
+    if (gb < nb_total) a.colsum[(static_cast<size_t>(bh) * nb_total + gb) * kD + d] = csum[bl][d];
   }
 }
 
@@ -683,19 +683,26 @@ static cudaError_t launch_tables(const ra_problem& p, int rot, float* ta, float*
 }
 
 // The three passes (channel reduce, finalize, quantise) for one input type and
-// rotation mode.
-template <bool kBf16, int kRot>
-static cudaError_t launch_passes(const PrologueArgs& a, dim3 grid, int red_bytes, int quant_bytes,
-                                 cudaStream_t st) {
+// rotation mode and head dimension.
+template <bool kBf16, int kRot, int kD>
+static cudaError_t launch_passes3(const PrologueArgs& a, dim3 grid, int red_bytes, int quant_bytes,
+                                  cudaStream_t st) {
   cudaError_t e;
-  if ((e = set_smem(prologue_reduce_kernel<kBf16, kRot>, red_bytes)) != cudaSuccess) return e;
-  prologue_reduce_kernel<kBf16, kRot><<<grid, kThreads, red_bytes, st>>>(a);
+  if ((e = set_smem(prologue_reduce_kernel<kBf16, kRot, kD>, red_bytes)) != cudaSuccess) return e;
+  prologue_reduce_kernel<kBf16, kRot, kD><<<grid, kThreads, red_bytes, st>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   prologue_finalize_kernel<<<grid.y, 128, 0, st>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if ((e = set_smem(prologue_quant_kernel<kBf16, kRot>, quant_bytes)) != cudaSuccess) return e;
-  prologue_quant_kernel<kBf16, kRot><<<grid, kThreads, quant_bytes, st>>>(a);
+  if ((e = set_smem(prologue_quant_kernel<kBf16, kRot, kD>, quant_bytes)) != cudaSuccess) return e;
+  prologue_quant_kernel<kBf16, kRot, kD><<<grid, kThreads, quant_bytes, st>>>(a);
   return cudaGetLastError();
+}
+
+template <bool kBf16, int kRot>
+static cudaError_t launch_passes(const PrologueArgs& a, dim3 grid, int red_bytes, int quant_bytes,
+                                 cudaStream_t st) {
+  return a.D == 128 ? launch_passes3<kBf16, kRot, 128>(a, grid, red_bytes, quant_bytes, st)
+                    : launch_passes3<kBf16, kRot, 64>(a, grid, red_bytes, quant_bytes, st);
 }
 
 cudaError_t launch_prologue(const ra_problem& p, int dtype, const void* q, const void* k, const void* v,
