@@ -281,6 +281,7 @@ __device__ __forceinline__ float group_max(float v, int lpt) {
 struct PrologueArgs {
   SegInfo s;
   int N, D, rot, dtype, block_k, nchunk;
+  int bk_log2;  // block_k = 2^bk_log2
   const void *q, *k, *v;
   const int32_t* pos;
   const float *tab_a, *tab_b;
@@ -505,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_quant_kernel(PrologueArg
   if (threadIdx.x == 0)
     for (int sc = 0; sc < kStg; ++sc) IO::issue(src, head, kD, a.N, n0, sc, stg, full);
   int cacc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-  int cblk = (warp * tpw) / a.block_k;  // key block of this warp's first tokens
+  int cblk = (warp * tpw) >> a.bk_log2;  // key block of this warp's first tokens
   // Adds this warp's per-thread column sums of block cblk to shared memory:
   // lanes holding the same channels (lpt apart) are combined first.
   auto flush = [&]() {
@@ -527,7 +528,7 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_quant_kernel(PrologueArg
     for (int ti = warp * tpw + tok_in_warp; ti - tok_in_warp < kSub; ti += step) {
       const int n = n0 + sc * kSub + ti;
       const bool valid = n < a.N;
-      const int blk = (sc * kSub + ti - tok_in_warp) / a.block_k;  // the same for the warp's tokens
+      const int blk = (sc * kSub + ti - tok_in_warp) >> a.bk_log2;  // the same for the warp's tokens
       if (blk != cblk) {
         flush();
         cblk = blk;
@@ -714,6 +715,7 @@ cudaError_t launch_prologue(const ra_problem& p, int dtype, const void* q, const
   PrologueArgs a;
   a.s = seg_info(p);
   a.N = p.N; a.D = p.D; a.rot = p.rot; a.dtype = dtype; a.block_k = p.block_k;
+  a.bk_log2 = __builtin_ctz(static_cast<unsigned>(p.block_k));
   a.nchunk = prologue_nchunk(p);
   a.q = q; a.k = k; a.v = v; a.pos = pos;
   a.tab_a = reinterpret_cast<float*>(base + w.tab_a);
@@ -752,6 +754,7 @@ cudaError_t launch_rope_bf16(const ra_problem& p, int dtype, const void* q, cons
   PrologueArgs a{};
   a.s = seg_info(p);
   a.N = p.N; a.D = p.D; a.rot = 0; a.dtype = dtype; a.block_k = p.block_k;
+  a.bk_log2 = __builtin_ctz(static_cast<unsigned>(p.block_k));
   a.nchunk = prologue_nchunk(p);
   a.q = q; a.k = k; a.pos = pos;
   a.tab_a = reinterpret_cast<float*>(base + w.tab_a);
