@@ -256,15 +256,21 @@ __device__ __forceinline__ void rope_apply8(const SegInfo& s, const RopePlan& rp
 }
 
 
-// Bits of 1.5 * 2^23 + clamp(rint(x * inv), -7, 7): clamping before rounding
-// gives the same integer (rint is monotone and +-7 are integers); the code is
-// the value minus 0x4B400000, and its low 4 bits are the two's complement nibble.
-__device__ __forceinline__ uint32_t quant4_bits(float x, float inv) {
-  const float y = fminf(fmaxf(__fmul_rn(x, inv), -7.0f), 7.0f);
-  return __float_as_uint(__fadd_rn(y, 12582912.0f));
+// For two elements: the bits of 1.5 * 2^23 + clamp(rint(x * inv), -7, 7).
+// Clamping before rounding gives the same integer (rint is monotone and +-7
+// are integers); the code is the value minus 0x4B400000, and its low 4 bits
+// are the two's complement nibble.  f32x2 arithmetic rounds each lane exactly
+// like the scalar operations.
+__device__ __forceinline__ void quant4_bits2(float x0, float x1, float inv0, float inv1, uint32_t* b) {
+  float2 y = __fmul2_rn(make_float2(x0, x1), make_float2(inv0, inv1));
+  y.x = fminf(fmaxf(y.x, -7.0f), 7.0f);
+  y.y = fminf(fmaxf(y.y, -7.0f), 7.0f);
+  const float2 t = __fadd2_rn(y, make_float2(12582912.0f, 12582912.0f));
+  b[0] = __float_as_uint(t.x);
+  b[1] = __float_as_uint(t.y);
 }
 
-// Packs the nibbles of eight quant4_bits results, element 2t in the low nibble.
+// Packs the nibbles of eight quant4_bits2 results, element 2t in the low nibble.
 __device__ __forceinline__ uint32_t pack8_bits(const uint32_t* b) {
   uint32_t p[4];
 #pragma unroll
@@ -565,10 +571,10 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_quant_kernel(PrologueArg
       const float iq = mq == 0.0f ? 0.0f : __fdiv_rn(7.0f, mq);
       const float ik = mk == 0.0f ? 0.0f : __fdiv_rn(7.0f, mk);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        bq[i] = quant4_bits(xq[i], iq);
-        bk[i] = quant4_bits(xk[i], ik);
-        bv[i] = quant4_bits(xv[i], vinv[i]);
+      for (int i = 0; i < 8; i += 2) {
+        quant4_bits2(xq[i], xq[i + 1], iq, iq, bq + i);
+        quant4_bits2(xk[i], xk[i + 1], ik, ik, bk + i);
+        quant4_bits2(xv[i], xv[i + 1], vinv[i], vinv[i + 1], bv + i);
       }
       if (valid) {
         const size_t o4 = head4 + static_cast<size_t>(n) * (kD / 2) + (c0 >> 1);
