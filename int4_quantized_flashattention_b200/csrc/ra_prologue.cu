@@ -72,7 +72,7 @@ __device__ __forceinline__ int grid_pos(const SegInfo& s, const int32_t* pos, in
 //   rot 1 (interleaved, fused table): y0 = x0 a + x1 b, y1 = x0 b - x1 a
 //   rot 0 / 2: y0 = x0 c - x1 s, y1 = x0 s + x1 c; rot 2 then pairs i, i + Dj/2
 //   through the per-warp row buffer `row` (D floats for this token).
-__device__ __forceinline__ void rope_rotate8(const SegInfo& s, const float* tab_a, const float* tab_b,
+__device__ __forceinline__ void rope_rotate8(const SegInfo& s, const float2* tab,
                                              const int32_t* pos, int n, int rot, int c0, float* x,
                                              float* row) {
 #pragma unroll
@@ -82,7 +82,8 @@ __device__ __forceinline__ void rope_rotate8(const SegInfo& s, const float* tab_
     const int k = (d - s.off[j]) >> 1;
     const int g = grid_pos(s, pos, n, j);
     const int idx = s.toff[j] + g * (s.dj[j] >> 1) + k;
-    const float a = __ldg(tab_a + idx), b = __ldg(tab_b + idx);
+    const float2 ab = __ldg(tab + idx);
+    const float a = ab.x, b = ab.y;
     const float x0 = x[2 * pr], x1 = x[2 * pr + 1];
     if (rot == 1) {
       x[2 * pr] = __fadd_rn(__fmul_rn(x0, a), __fmul_rn(x1, b));
@@ -175,8 +176,8 @@ struct RopePlan {
 // Table coefficients (a, b) of the thread's 4 channel pairs for a token at grid
 // position gp (one position per segment; out-of-grid positions are reported
 // and clamped so every table access stays in bounds).
-__device__ __forceinline__ void rope_coef8p(const SegInfo& s, const RopePlan& rp, const float* tab_a,
-                                            const float* tab_b, const int* gp, float* ca, float* cb) {
+__device__ __forceinline__ void rope_coef8p(const SegInfo& s, const RopePlan& rp, const float2* tab,
+                                            const int* gp, float* ca, float* cb) {
   int g[3];
 #pragma unroll
   for (int j = 0; j < 3; ++j) {
@@ -190,8 +191,9 @@ __device__ __forceinline__ void rope_coef8p(const SegInfo& s, const RopePlan& rp
   for (int pr = 0; pr < 4; ++pr) {
     const int gj = rp.seg[pr] == 0 ? g[0] : (rp.seg[pr] == 1 ? g[1] : g[2]);
     const int idx = rp.off[pr] + gj * rp.stride[pr];
-    ca[pr] = __ldg(tab_a + idx);
-    cb[pr] = __ldg(tab_b + idx);
+    const float2 ab = __ldg(tab + idx);
+    ca[pr] = ab.x;
+    cb[pr] = ab.y;
   }
 }
 
@@ -290,7 +292,7 @@ struct PrologueArgs {
   int bk_log2;  // block_k = 2^bk_log2
   const void *q, *k, *v;
   const int32_t* pos;
-  const float *tab_a, *tab_b;
+  const float2* tab;   // RoPE table entries (a, b)
   double* ksum;     // [BH, nchunk, D]
   float* vmax;      // [BH, nchunk, D]
   float* vinv;      // [BH, D]
@@ -301,7 +303,7 @@ struct PrologueArgs {
 
 // Table entry e -> (segment j, position g, pair k); angle g * theta^(-2k/Dj) in
 // fp64, entries rounded once to fp32.  rot 1 stores the fused H2 block.
-__global__ void rope_table_kernel(SegInfo s, int total, double theta, int rot, float* tab_a, float* tab_b) {
+__global__ void rope_table_kernel(SegInfo s, int total, double theta, int rot, float2* tab) {
   const int e = blockIdx.x * blockDim.x + threadIdx.x;
   if (e >= total) return;
   const int j = e < s.toff[1] ? 0 : (e < s.toff[2] ? 1 : 2);
@@ -311,11 +313,9 @@ __global__ void rope_table_kernel(SegInfo s, int total, double theta, int rot, f
   const double phi = static_cast<double>(g) * freq;
   const double c = cos(phi), sn = sin(phi);
   if (rot == 1) {
-    tab_a[e] = static_cast<float>((c + sn) / sqrt(2.0));
-    tab_b[e] = static_cast<float>((c - sn) / sqrt(2.0));
+    tab[e] = make_float2(static_cast<float>((c + sn) / sqrt(2.0)), static_cast<float>((c - sn) / sqrt(2.0)));
   } else {
-    tab_a[e] = static_cast<float>(c);
-    tab_b[e] = static_cast<float>(sn);
+    tab[e] = make_float2(static_cast<float>(c), static_cast<float>(sn));
   }
 }
 
@@ -416,7 +416,7 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_reduce_kernel(PrologueAr
         for (int i = 0; i < 8; ++i) { x[i] = 0.0f; y[i] = 0.0f; }
       }
       // Every lane takes part (the half rotation synchronises the warp).
-      rope_coef8p(a.s, rp, a.tab_a, a.tab_b, gp, ca, cb);
+      rope_coef8p(a.s, rp, a.tab, gp, ca, cb);
       rope_apply8(a.s, rp, kRot, ca, cb, c0, x, rows[warp][tok_in_warp]);
       if (valid) {
 #pragma unroll
@@ -555,7 +555,7 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_quant_kernel(PrologueArg
 #pragma unroll
         for (int i = 0; i < 8; ++i) { xq[i] = 0.0f; xk[i] = 0.0f; xv[i] = 0.0f; }
       }
-      rope_coef8p(a.s, rp, a.tab_a, a.tab_b, gp, ca, cb);
+      rope_coef8p(a.s, rp, a.tab, gp, ca, cb);
       rope_apply8(a.s, rp, kRot, ca, cb, c0, xq, rows[warp][tok_in_warp]);
       rope_apply8(a.s, rp, kRot, ca, cb, c0, xk, rows[warp][tok_in_warp]);
       float mq = 0.0f, mk = 0.0f;
@@ -623,7 +623,7 @@ __global__ void __launch_bounds__(kThreads) rope_bf16_kernel(PrologueArgs a, __n
 #pragma unroll
     for (int which = 0; which < 2; ++which) {
       load8(which ? a.k : a.q, head + static_cast<size_t>(n) * a.D + c0, a.dtype, x);
-      rope_rotate8(a.s, a.tab_a, a.tab_b, a.pos, n, 0, c0, x, rows[warp][tok_in_warp]);
+      rope_rotate8(a.s, a.tab, a.pos, n, 0, c0, x, rows[warp][tok_in_warp]);
       uint32_t w[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -668,8 +668,7 @@ WorkspaceLayout workspace_layout(const ra_problem& p) {
   WorkspaceLayout w;
   const size_t bh = static_cast<size_t>(p.B) * p.H, T = rope_table_len(p), nc = prologue_nchunk(p);
   size_t o = 0;
-  w.tab_a = o; o = align256(o + T * sizeof(float));
-  w.tab_b = o; o = align256(o + T * sizeof(float));
+  w.tab = o; o = align256(o + T * sizeof(float2));
   w.ksum = o;  o = align256(o + bh * nc * p.D * sizeof(double));
   w.vmax = o;  o = align256(o + bh * nc * p.D * sizeof(float));
   w.vinv = o;  o = align256(o + bh * p.D * sizeof(float));
@@ -682,10 +681,10 @@ static cudaError_t set_smem(K kern, int bytes) {
   return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
-static cudaError_t launch_tables(const ra_problem& p, int rot, float* ta, float* tb, cudaStream_t st) {
+static cudaError_t launch_tables(const ra_problem& p, int rot, float2* tab, cudaStream_t st) {
   const SegInfo s = seg_info(p);
   const int T = static_cast<int>(rope_table_len(p));
-  rope_table_kernel<<<(T + 255) / 256, 256, 0, st>>>(s, T, static_cast<double>(p.theta), rot, ta, tb);
+  rope_table_kernel<<<(T + 255) / 256, 256, 0, st>>>(s, T, static_cast<double>(p.theta), rot, tab);
   return cudaGetLastError();
 }
 
@@ -724,14 +723,13 @@ cudaError_t launch_prologue(const ra_problem& p, int dtype, const void* q, const
   a.bk_log2 = __builtin_ctz(static_cast<unsigned>(p.block_k));
   a.nchunk = prologue_nchunk(p);
   a.q = q; a.k = k; a.v = v; a.pos = pos;
-  a.tab_a = reinterpret_cast<float*>(base + w.tab_a);
-  a.tab_b = reinterpret_cast<float*>(base + w.tab_b);
+  a.tab = reinterpret_cast<const float2*>(base + w.tab);
   a.ksum = reinterpret_cast<double*>(base + w.ksum);
   a.vmax = reinterpret_cast<float*>(base + w.vmax);
   a.vinv = reinterpret_cast<float*>(base + w.vinv);
   a.q4 = q4; a.k4 = k4; a.v4 = v4; a.sq = sq; a.sk = sk; a.k_mean = k_mean; a.sv = sv;
   a.colsum = colsum;
-  cudaError_t e = launch_tables(p, p.rot, const_cast<float*>(a.tab_a), const_cast<float*>(a.tab_b), st);
+  cudaError_t e = launch_tables(p, p.rot, reinterpret_cast<float2*>(base + w.tab), st);
   if (e != cudaSuccess) return e;
   const dim3 grid(a.nchunk, p.B * p.H);
   // Dynamic shared memory: kStg staged sub-chunks (the reduce pass reuses it
@@ -763,9 +761,8 @@ cudaError_t launch_rope_bf16(const ra_problem& p, int dtype, const void* q, cons
   a.bk_log2 = __builtin_ctz(static_cast<unsigned>(p.block_k));
   a.nchunk = prologue_nchunk(p);
   a.q = q; a.k = k; a.pos = pos;
-  a.tab_a = reinterpret_cast<float*>(base + w.tab_a);
-  a.tab_b = reinterpret_cast<float*>(base + w.tab_b);
-  cudaError_t e = launch_tables(p, 0, const_cast<float*>(a.tab_a), const_cast<float*>(a.tab_b), st);
+  a.tab = reinterpret_cast<const float2*>(base + w.tab);
+  cudaError_t e = launch_tables(p, 0, reinterpret_cast<float2*>(base + w.tab), st);
   if (e != cudaSuccess) return e;
   rope_bf16_kernel<<<dim3(a.nchunk, p.B * p.H), kThreads, 0, st>>>(a, static_cast<__nv_bfloat16*>(qo),
                                                                    static_cast<__nv_bfloat16*>(ko));
