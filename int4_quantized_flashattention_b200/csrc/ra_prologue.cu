@@ -461,10 +461,26 @@ __global__ void prologue_finalize_kernel(PrologueArgs a) {
   if (d >= a.D) return;
   double sum = 0.0;
   float mx = 0.0f;
-  for (int c = 0; c < a.nchunk; ++c) {
-    const size_t o = (static_cast<size_t>(bh) * a.nchunk + c) * a.D + d;
-    sum += a.ksum[o];
-    mx = fmaxf(mx, a.vmax[o]);
+  const size_t o0 = static_cast<size_t>(bh) * a.nchunk * a.D + d;
+  int c = 0;
+  // Eight chunks' loads in flight at a time; the sum keeps the chunk order.
+  for (; c + 8 <= a.nchunk; c += 8) {
+    double s8[8];
+    float m8[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      s8[u] = a.ksum[o0 + static_cast<size_t>(c + u) * a.D];
+      m8[u] = a.vmax[o0 + static_cast<size_t>(c + u) * a.D];
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      sum += s8[u];
+      mx = fmaxf(mx, m8[u]);
+    }
+  }
+  for (; c < a.nchunk; ++c) {
+    sum += a.ksum[o0 + static_cast<size_t>(c) * a.D];
+    mx = fmaxf(mx, a.vmax[o0 + static_cast<size_t>(c) * a.D]);
   }
   a.k_mean[bh * a.D + d] = static_cast<float>(sum / static_cast<double>(a.N));
   a.sv[bh * a.D + d] = __fdiv_rn(mx, 7.0f);
