@@ -324,9 +324,12 @@ __global__ void rope_table_kernel(SegInfo s, int total, double theta, int rot, f
 // each SM keeps tens of kilobytes of loads in flight.  Thread 0 issues the
 // copies; every stage has one mbarrier that completes on the copied bytes.
 constexpr int kSub = 32;   // tokens per stage
-constexpr int kStg = 2;    // stages
+// Two stages per pass: more stages in flight (4 or 6 for the reduce pass, 3
+// for the quantise pass at two CTAs per SM) measured no faster.
+constexpr int kStgR = 2;   // stages of the channel-reduce pass (K, V)
+constexpr int kStgQ = 2;   // stages of the quantise pass (Q, K, V)
 
-template <bool kBf16, int NT>
+template <bool kBf16, int NT, int kStg>
 struct StageIO {
   static constexpr int kEl = kBf16 ? 2 : 4;
   // Issues the copies of sub-chunk sc (tokens n0 + sc*kSub ...) of NT tensors
@@ -367,15 +370,17 @@ __device__ __forceinline__ bool stage_wait(uint64_t* bar, uint32_t parity, volat
 // mode keeps only its own per-thread state).
 template <bool kBf16, int kRot, int kD>
 __global__ void __launch_bounds__(kThreads, 3) prologue_reduce_kernel(PrologueArgs a) {
-  using IO = StageIO<kBf16, 2>;
-  __shared__ float rows[kThreads / 32][4][128];
-  __shared__ uint64_t full[kStg];
+  using IO = StageIO<kBf16, 2, kStgR>;
+  // Row buffer of the half rotation's exchange (one token row per warp slot).
+  __shared__ float rows[kRot == 2 ? kThreads / 32 : 1][4][128];
+  __shared__ uint64_t full[kStgR];
   __shared__ int abort_flag;
   extern __shared__ __align__(128) uint8_t stg[];
   const int bh = blockIdx.y, chunk = blockIdx.x;
   const int lpt = kD >> 3, tpw = 32 / lpt;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tok_in_warp = lane / lpt, c0 = (lane % lpt) * 8;
+  float* const row = rows[kRot == 2 ? warp : 0][kRot == 2 ? tok_in_warp : 0];
   const int step = (kThreads / 32) * tpw;
   const int n0 = chunk * kChunk;
   const size_t head = static_cast<size_t>(bh) * a.N * kD;
@@ -383,21 +388,21 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_reduce_kernel(PrologueAr
   RopePlan rp;
   rp.init(a.s, c0);
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStg; ++s) mbar_init(full + s, 1);
+    for (int s = 0; s < kStgR; ++s) mbar_init(full + s, 1);
     abort_flag = 0;
     fence_barrier_init();
   }
   __syncthreads();
   if (threadIdx.x == 0)
-    for (int sc = 0; sc < kStg; ++sc) IO::issue(src, head, kD, a.N, n0, sc, stg, full);
+    for (int sc = 0; sc < kStgR; ++sc) IO::issue(src, head, kD, a.N, n0, sc, stg, full);
   double ks[8];
   float vm[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) { ks[i] = 0.0; vm[i] = 0.0f; }
   bool ok = true;
   for (int sc = 0; sc < kChunk / kSub && ok; ++sc) {
-    const int s = sc % kStg;
-    if (!(ok = stage_wait(full + s, (sc / kStg) & 1, &abort_flag))) break;
+    const int s = sc % kStgR;
+    if (!(ok = stage_wait(full + s, (sc / kStgR) & 1, &abort_flag))) break;
     for (int ti = warp * tpw + tok_in_warp; ti - tok_in_warp < kSub; ti += step) {
       const int n = n0 + sc * kSub + ti;
       const bool valid = n < a.N;
@@ -417,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_reduce_kernel(PrologueAr
       }
       // Every lane takes part (the half rotation synchronises the warp).
       rope_coef8p(a.s, rp, a.tab, gp, ca, cb);
-      rope_apply8(a.s, rp, kRot, ca, cb, c0, x, rows[warp][tok_in_warp]);
+      rope_apply8(a.s, rp, kRot, ca, cb, c0, x, row);
       if (valid) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -427,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_reduce_kernel(PrologueAr
       }
     }
     __syncthreads();  // stage s consumed
-    if (threadIdx.x == 0 && sc + kStg < kChunk / kSub) IO::issue(src, head, kD, a.N, n0, sc + kStg, stg, full);
+    if (threadIdx.x == 0 && sc + kStgR < kChunk / kSub) IO::issue(src, head, kD, a.N, n0, sc + kStgR, stg, full);
   }
   if (!ok) {
     if (threadIdx.x == 0) atomicOr(&g_prologue_status, kStatusTimeout);
@@ -494,16 +499,18 @@ __global__ void prologue_finalize_kernel(PrologueArgs a) {
 // memory.
 template <bool kBf16, int kRot, int kD>
 __global__ void __launch_bounds__(kThreads, 3) prologue_quant_kernel(PrologueArgs a) {
-  using IO = StageIO<kBf16, 3>;
-  __shared__ float rows[kThreads / 32][4][128];
+  using IO = StageIO<kBf16, 3, kStgQ>;
+  // Row buffer of the half rotation's exchange (one token row per warp slot).
+  __shared__ float rows[kRot == 2 ? kThreads / 32 : 1][4][128];
   __shared__ int csum[kChunk / 16][128];
-  __shared__ uint64_t full[kStg];
+  __shared__ uint64_t full[kStgQ];
   __shared__ int abort_flag;
   extern __shared__ __align__(128) uint8_t stg[];
   const int bh = blockIdx.y, chunk = blockIdx.x;
   const int lpt = kD >> 3, tpw = 32 / lpt;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tok_in_warp = lane / lpt, c0 = (lane % lpt) * 8;
+  float* const row = rows[kRot == 2 ? warp : 0][kRot == 2 ? tok_in_warp : 0];
   const int step = (kThreads / 32) * tpw;
   const int nblk = kChunk / a.block_k;
   const int n0 = chunk * kChunk;
@@ -514,7 +521,7 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_quant_kernel(PrologueArg
   rp.init(a.s, c0);
   for (int i = threadIdx.x; i < nblk * kD; i += kThreads) csum[i / kD][i % kD] = 0;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStg; ++s) mbar_init(full + s, 1);
+    for (int s = 0; s < kStgQ; ++s) mbar_init(full + s, 1);
     abort_flag = 0;
     fence_barrier_init();
   }
@@ -526,7 +533,7 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_quant_kernel(PrologueArg
   }
   __syncthreads();
   if (threadIdx.x == 0)
-    for (int sc = 0; sc < kStg; ++sc) IO::issue(src, head, kD, a.N, n0, sc, stg, full);
+    for (int sc = 0; sc < kStgQ; ++sc) IO::issue(src, head, kD, a.N, n0, sc, stg, full);
   int cacc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   int cblk = (warp * tpw) >> a.bk_log2;  // key block of this warp's first tokens
   // Adds this warp's per-thread column sums of block cblk to shared memory:
@@ -545,8 +552,8 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_quant_kernel(PrologueArg
   };
   bool ok = true;
   for (int sc = 0; sc < kChunk / kSub && ok; ++sc) {
-    const int s = sc % kStg;
-    if (!(ok = stage_wait(full + s, (sc / kStg) & 1, &abort_flag))) break;
+    const int s = sc % kStgQ;
+    if (!(ok = stage_wait(full + s, (sc / kStgQ) & 1, &abort_flag))) break;
     for (int ti = warp * tpw + tok_in_warp; ti - tok_in_warp < kSub; ti += step) {
       const int n = n0 + sc * kSub + ti;
       const bool valid = n < a.N;
@@ -572,8 +579,8 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_quant_kernel(PrologueArg
         for (int i = 0; i < 8; ++i) { xq[i] = 0.0f; xk[i] = 0.0f; xv[i] = 0.0f; }
       }
       rope_coef8p(a.s, rp, a.tab, gp, ca, cb);
-      rope_apply8(a.s, rp, kRot, ca, cb, c0, xq, rows[warp][tok_in_warp]);
-      rope_apply8(a.s, rp, kRot, ca, cb, c0, xk, rows[warp][tok_in_warp]);
+      rope_apply8(a.s, rp, kRot, ca, cb, c0, xq, row);
+      rope_apply8(a.s, rp, kRot, ca, cb, c0, xk, row);
       float mq = 0.0f, mk = 0.0f;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -606,7 +613,7 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_quant_kernel(PrologueArg
       }
     }
     __syncthreads();  // stage s consumed
-    if (threadIdx.x == 0 && sc + kStg < kChunk / kSub) IO::issue(src, head, kD, a.N, n0, sc + kStg, stg, full);
+    if (threadIdx.x == 0 && sc + kStgQ < kChunk / kSub) IO::issue(src, head, kD, a.N, n0, sc + kStgQ, stg, full);
   }
   if (!ok) {
     if (threadIdx.x == 0) atomicOr(&g_prologue_status, kStatusTimeout);
@@ -748,11 +755,11 @@ cudaError_t launch_prologue(const ra_problem& p, int dtype, const void* q, const
   cudaError_t e = launch_tables(p, p.rot, reinterpret_cast<float2*>(base + w.tab), st);
   if (e != cudaSuccess) return e;
   const dim3 grid(a.nchunk, p.B * p.H);
-  // Dynamic shared memory: kStg staged sub-chunks (the reduce pass reuses it
+  // Dynamic shared memory: the staged sub-chunks (the reduce pass reuses it
   // for its per-thread partial sums, 12 bytes x 8 channels x threads).
   const int el = dtype == 1 ? 2 : 4;
-  const int red_bytes = kStg * 2 * kSub * p.D * el > kThreads * 8 * 12 ? kStg * 2 * kSub * p.D * el : kThreads * 8 * 12;
-  const int quant_bytes = kStg * 3 * kSub * p.D * el;
+  const int red_bytes = kStgR * 2 * kSub * p.D * el > kThreads * 8 * 12 ? kStgR * 2 * kSub * p.D * el : kThreads * 8 * 12;
+  const int quant_bytes = kStgQ * 3 * kSub * p.D * el;
   switch (dtype * 4 + p.rot) {
 #define RA_PRO(DT, ROT)                                                                              \
   case DT * 4 + ROT:                                                                                 \
