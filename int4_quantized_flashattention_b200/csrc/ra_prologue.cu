@@ -403,6 +403,8 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_reduce_kernel(PrologueAr
   for (int sc = 0; sc < kChunk / kSub && ok; ++sc) {
     const int s = sc % kStgR;
     if (!(ok = stage_wait(full + s, (sc / kStgR) & 1, &abort_flag))) break;
+    // Two tokens per thread in flight (latency of the position and table loads).
+#pragma unroll 2
     for (int ti = warp * tpw + tok_in_warp; ti - tok_in_warp < kSub; ti += step) {
       const int n = n0 + sc * kSub + ti;
       const bool valid = n < a.N;
@@ -554,6 +556,9 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_quant_kernel(PrologueArg
   for (int sc = 0; sc < kChunk / kSub && ok; ++sc) {
     const int s = sc % kStgQ;
     if (!(ok = stage_wait(full + s, (sc / kStgQ) & 1, &abort_flag))) break;
+    // Two tokens per thread in flight: independent work to hide the latency
+    // of the position and table loads and of the shuffles.
+#pragma unroll 2
     for (int ti = warp * tpw + tok_in_warp; ti - tok_in_warp < kSub; ti += step) {
       const int n = n0 + sc * kSub + ti;
       const bool valid = n < a.N;
