@@ -43,6 +43,9 @@
  *      SageAttention-style codes c = rint(7 exp(S - m)) in [0, 7] with no zero
  *      point, dequantised as c / 7; l_mode FP32 makes the denominator the
  *      plain sum of exp(S - m_codes) instead of the dequantised code sum.
+ *   R12 The full rotation (rot 3) is RoPE followed by the row times H_D /
+ *      sqrt(D), H_D the Sylvester Hadamard matrix, evaluated as butterflies
+ *      at distances 1, 2, ..., D/2 in fp32 and one final scaling.
  *   R10 Codes are packed two per byte, element 2t in the low nibble, as
  *      4-bit two's complement.
  */
