@@ -412,6 +412,11 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     // instruction, each rounded exactly like the scalar form).
     const float2 kNegMagic2 = make_float2(-kMagicF, -kMagicF);
     const float2 kMagic2 = make_float2(kMagicF, kMagicF);
+    // Byte-lane magics: fp32 values in [2^23, 2^24) with a zero low byte whose
+    // bits K0..K3 satisfy K0 + K1 2^8 + K2 2^16 + K3 2^24 = 0 mod 2^32, so
+    // t0 + t1 2^8 + t2 2^16 + t3 2^24 of the rounded sums is the packed word.
+    const float2 kMagLo = make_float2(8388608.0f, 11862016.0f);   // bits 0x4B000000, 0x4B350000
+    const float2 kMagHi = make_float2(8421376.0f, kMagicF);       // bits 0x4B008000, 0x4B400000
     constexpr int kPMode = MODE & 3;
     constexpr bool kLf = (MODE & 4) != 0;
     constexpr float kLevels = kPMode == 2 ? 7.0f : 15.0f;  // code for P = 1
@@ -526,8 +531,9 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const bool grow = m_new > m_run;
         const float Mp = __fmul_rn(kPMode == 1 ? m_blk : m_new, kLog2e);  // the max the codes use
         const float2 nMp2 = make_float2(-Mp, -Mp);
-        // P code c + 8 = rint(15 exp2(y)): adding 15 e to 1.5 * 2^23 rounds it
-        // to an integer that lands in the low byte of the sum's bits.
+        // P code c + 8 = rint(15 exp2(y)): adding 15 e to a magic in [2^23, 2^24)
+        // with a zero low byte rounds it to an integer that lands in the low
+        // byte of the sum's bits.
         uint32_t words[kHK / 4];
         float2 esum = make_float2(0.0f, 0.0f);
 #pragma unroll
@@ -536,8 +542,8 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           const float2 x23 = __ffma2_rn(v2[2 * q + 1], cpi2, nMp2);
           float2 e01 = make_float2(ex2_approx(x01.x), ex2_approx(x01.y));
           float2 e23 = make_float2(ex2_approx(x23.x), ex2_approx(x23.y));
-          const float2 t01 = __ffma2_rn(kLv2, e01, kMagic2);
-          const float2 t23 = __ffma2_rn(kLv2, e23, kMagic2);
+          const float2 t01 = __ffma2_rn(kLv2, e01, kMagLo);
+          const float2 t23 = __ffma2_rn(kLv2, e23, kMagHi);
           if constexpr (kLf) {
             if (nvalid < BN) {  // keys past N (NaN scores) do not count
               const int j = hh * kHK + 4 * q;
@@ -546,8 +552,12 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             }
             esum = __fadd2_rn(esum, __fadd2_rn(e01, e23));
           }
-          words[q] = __byte_perm(__byte_perm(__float_as_uint(t01.x), __float_as_uint(t01.y), 0x0040),
-                                 __byte_perm(__float_as_uint(t23.x), __float_as_uint(t23.y), 0x0040), 0x5410);
+          // Integer multiply-adds (FMA pipe) instead of byte permutes (ALU).
+          // Keys past N give NaN bits; they form a suffix of the word, and
+          // the carries of their garbage only reach higher (also masked) bytes.
+          const uint32_t lo = __float_as_uint(t01.y) * 256u + __float_as_uint(t01.x);
+          const uint32_t hi = __float_as_uint(t23.y) * 256u + __float_as_uint(t23.x);
+          words[q] = hi * 65536u + lo;
         }
         if (nvalid < BN) {  // last, ragged block: codes of keys past N are 0
 #pragma unroll
