@@ -262,6 +262,21 @@ def test_full_size_sampled(ra, dev, orc, name, heads, tiles):
     assert tc.end_to_end() <= 1e-3, (tc.end_to_end(), tc.flips, tc.relevant)
 
 
+def test_full_size_sampled_ablations(ra, dev, orc):
+    """The ablation modes bench.py times, at the wan size it times them: sampled
+    tiles against the oracle's switches."""
+    wl = si.WORKLOADS["wan"]
+    x = si.make_inputs(wl)
+    tiles = ((0, 0), (13, 77), (27, 200), (39, 255))
+    for p_mode, l_mode in ((1, 0), (2, 1), (0, 1)):
+        p, codes, host = gu.gpu_forward(ra, wl, x, dev, with_lse=True, p_mode=p_mode, l_mode=l_mode)
+        assert np.all(np.isfinite(host["out"])) and np.all(np.isfinite(host["lse"]))
+        tc = TileCheck(ra, orc, wl, p, codes, host, p_mode=p_mode, l_mode=l_mode)
+        for h, t in tiles:
+            tc.tile(h, t)
+        assert tc.end_to_end() <= 1e-3, (p_mode, l_mode, tc.end_to_end(), tc.flips, tc.relevant)
+
+
 def test_repeat_runs_are_bitwise_identical(ra, dev):
     """The kernel is deterministic (flush decisions and accumulation order depend
     only on the data), so repeated runs must agree bit for bit; any difference
