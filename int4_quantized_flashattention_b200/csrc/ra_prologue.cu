@@ -1,7 +1,9 @@
 // Fused prologue of the RotateAttention INT4 forward (memory-bound):
 //   3D RoPE + RoPE-aware rotation of Q and K, K smoothing, per-token INT4 of Q
 //   and K, per-channel INT4 of V and per-block V column sums; plus the plain
-//   RoPE to bf16 that feeds the bf16 fallback.
+//   RoPE to bf16 that feeds the bf16 fallback.  Rotation modes: interleaved
+//   (H2 fused into the RoPE table), half (pairs i, i + Dj/2), full (the row
+//   times a D x D Hadamard matrix), none.
 // Method: RotateAttention (arXiv 2607.02584), papernotes page "overall
 // framework" and "key design 1"; gecl notes "Key Insight" (per-token INT4).
 //
@@ -9,8 +11,9 @@
 // round-to-nearest intrinsics in a fixed order (no contraction), so codes
 // match an fp32 reference of the same definition bit for bit.
 //
-// Layout: 8 consecutive channels per thread, D/8 threads per token, so a warp
-// reads 512 contiguous bytes of bf16 per token pair with 16-byte loads.
+// Layout: token rows are staged in shared memory by bulk copies; a thread
+// works on 8 consecutive channels of a token (D/8 threads per token, 16-byte
+// shared-memory reads).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
