@@ -411,7 +411,6 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     // Arithmetic on pairs of fp32 (sm_100 f32x2 instructions: two lanes per
     // instruction, each rounded exactly like the scalar form).
     const float2 kNegMagic2 = make_float2(-kMagicF, -kMagicF);
-    const float2 kMagic2 = make_float2(kMagicF, kMagicF);
     // Byte-lane magics: fp32 values in [2^23, 2^24) with a zero low byte whose
     // bits K0..K3 satisfy K0 + K1 2^8 + K2 2^16 + K3 2^24 = 0 mod 2^32, so
     // t0 + t1 2^8 + t2 2^16 + t3 2^24 of the rounded sums is the packed word.
