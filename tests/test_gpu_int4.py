@@ -323,3 +323,27 @@ def test_ablation_switches_change_the_result(ra, dev, orc):
     for key, o in outs.items():
         if key != (0, 0):
             assert gu.rel_l2(o, base) > 1e-3, key
+
+
+def test_batch_of_two(ra, dev, orc):
+    """B = 2: every (batch, head) is its own problem in the flat head index of
+    the prologue, the attention and the test entry."""
+    wl = si.WORKLOADS["small"].with_(name="small_b2", B=2)
+    x = si.make_inputs(wl)
+    p, codes, host = gu.gpu_forward(ra, wl, x, dev, with_lse=True)
+    po = orc.problem(wl)
+    for b in range(wl.B):
+        for h in range(wl.H):
+            ref = orc.prologue_head(po, x["q"][b, h], x["k"][b, h], x["v"][b, h], x["pos"])
+            for name in ("q4", "k4", "v4"):
+                frac, mx = gu.code_agreement(host[name][b, h], ref[name], orc)
+                assert frac >= CODE_EXACT and mx <= 1, (b, h, name, frac, mx)
+            out = orc.attention_int4_rows(po, ref, 0, wl.N)["out"]
+            assert gu.rel_l2(host["out"][b, h], gu.bf16_round(out)) <= 1e-3, (b, h)
+    # the test entry addresses (batch 1, head 1): S_int of its first tile
+    _, _, s, _, _ = ra.test_int4_codes(p, codes, 1, 1, 0)
+    assert ra.sync_status() == 0
+    hc = gu.head_codes(host, (1, 1))
+    R = min(128, wl.N)
+    ref = orc.attention_int4_rows(po, hc, 0, R, dumps=True)
+    assert np.array_equal(s.cpu().numpy()[:R], ref["s_int"])
