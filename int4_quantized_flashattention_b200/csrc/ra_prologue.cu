@@ -599,15 +599,8 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_quant_kernel(PrologueArg
       mq = group_max(mq, lpt);
       mk = group_max(mk, lpt);
       uint32_t bq[8], bk[8], bv[8];
-      // One IEEE division per lane instead of four: even lanes of the token
-      // divide for Q, odd lanes for K, and the pair exchanges by shuffles;
-      // 7/amax and amax/7 likewise (the scales are stored by lanes 0 and 1).
-      const int li = c0 >> 3;
-      const float am = (li & 1) ? mk : mq;
-      const float rcp7 = __fdiv_rn(7.0f, am);
-      const float s7 = __fdiv_rn(am, 7.0f);
-      const float iq = mq == 0.0f ? 0.0f : __shfl_sync(0xFFFFFFFFu, rcp7, lane & ~1);
-      const float ik = mk == 0.0f ? 0.0f : __shfl_sync(0xFFFFFFFFu, rcp7, lane | 1);
+      const float iq = mq == 0.0f ? 0.0f : __fdiv_rn(7.0f, mq);
+      const float ik = mk == 0.0f ? 0.0f : __fdiv_rn(7.0f, mk);
 #pragma unroll
       for (int i = 0; i < 8; i += 2) {
         quant4_bits2(xq[i], xq[i + 1], iq, iq, bq + i);
@@ -619,7 +612,10 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_quant_kernel(PrologueArg
         *reinterpret_cast<uint32_t*>(a.q4 + o4) = pack8_bits(bq);
         *reinterpret_cast<uint32_t*>(a.k4 + o4) = pack8_bits(bk);
         *reinterpret_cast<uint32_t*>(a.v4 + o4) = pack8_bits(bv);
-        if (li < 2) (li == 0 ? a.sq : a.sk)[static_cast<size_t>(bh) * a.N + n] = s7;
+        if (c0 == 0) {
+          a.sq[static_cast<size_t>(bh) * a.N + n] = __fdiv_rn(mq, 7.0f);
+          a.sk[static_cast<size_t>(bh) * a.N + n] = __fdiv_rn(mk, 7.0f);
+        }
 #pragma unroll
         for (int i = 0; i < 8; ++i) cacc[i] += static_cast<int>(bv[i] - 0x4B400000u);
       }
