@@ -19,7 +19,7 @@
  * Everything else (channel means, the attention accumulators, the reference
  * attention) is fp64.
  *
- * Readings of points the pages leave open (each is listed in the design doc):
+ * Readings of points the pages leave open:
  *   R1 RoPE pairs are adjacent channels (2k, 2k+1) of a segment; the segment's
  *      frequencies are theta^(-2k/Dj); rotation by angle p*freq is the complex
  *      product (x0 + i x1) e^{i phi}.
