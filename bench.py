@@ -96,7 +96,7 @@ def _workload(name):
 
 
 def _config(wl, extra=None):
-    rot = {0: "none", 1: "interleaved", 2: "half"}[wl.rot]
+    rot = {0: "none", 1: "interleaved", 2: "half", 3: "full"}[wl.rot]
     c = {"workload": f"{wl.name}: B={wl.B} H={wl.H} N={wl.N} (grid {wl.grid[0]}x{wl.grid[1]}x{wl.grid[2]}) "
                      f"D={wl.D} seg={wl.seg[0]}/{wl.seg[1]}/{wl.seg[2]} rot={rot} blocks {wl.block_q}x{wl.block_k}",
          "B": wl.B, "H": wl.H, "N": wl.N, "D": wl.D, "seg": list(wl.seg), "rot": rot,
