@@ -615,8 +615,10 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         // maximum); reset A when its magnitude bound nears the exact range of
         // the read-back (|A| < 2^22).
         const bool near_bound = (Labs + 15 * BN) * 112 >= (1 << 22) - 4096;
+        // Both votes are taken by every lane before either is used.
         const bool reset = __any_sync(0xFFFFFFFFu, (t > 0) && (near_bound || DUMP));
-        if (reset || __any_sync(0xFFFFFFFFu, (t > 0) && change)) {
+        const bool any_change = __any_sync(0xFFFFFFFFu, (t > 0) && change);
+        if (reset || any_change) {
           if (!(ok = wait_at(B.pv_done + tt * 2 + ((g - 1) & 1), ((g - 1) >> 1) & 1, abort_flag, 12u, g))) break;
           __syncwarp();
           tc_fence_after();

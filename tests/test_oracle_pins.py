@@ -204,6 +204,35 @@ def test_qk_quantisation_round_trip(orc, name):
         assert np.allclose(s, np.abs(xr).max(axis=1) / 7.0, rtol=1e-6)
 
 
+@pytest.mark.parametrize("name", ["tiny", "small"])
+def test_v_quantisation_round_trip(orc, name):
+    """Per-channel symmetric INT4 of V (papernotes page, overall framework:
+    quantised V; the same symmetric rule as Q and K, taken over the tokens of a
+    channel): codes in [-7, 7], |v - s_v c| <= s_v/2 for every element, the
+    largest magnitude of each channel maps to +-7 with the value's sign, and
+    s_v = amax/7 of its own channel.  Floor instead of rint, a missing clamp
+    or a scale taken from another channel each breaks one of these."""
+    wl, p, x, h = _head(orc, name)
+    v = x["v"][0, 0].astype(np.float64)
+    c = orc.unpack_codes(h["v4"]).astype(np.float64)
+    s = h["sv"].astype(np.float64)
+    assert c.min() >= -7 and c.max() <= 7
+    err = np.abs(v - s[None, :] * c)
+    assert np.all(err <= s[None, :] * 0.5 * (1 + 1e-5) + 1e-7)
+    amax_idx = np.abs(v).argmax(axis=0)
+    top = c[amax_idx, np.arange(wl.D)]
+    assert np.all(top == 7 * np.sign(v[amax_idx, np.arange(wl.D)]))
+    assert np.allclose(s, np.abs(v).max(axis=0) / 7.0, rtol=1e-6)
+    # channels are quantised independently: scaling one channel of V by 2
+    # doubles its scale and leaves every code unchanged
+    v2 = x["v"][0, 0].copy()
+    v2[:, 3] *= 2.0
+    h2 = orc.prologue_head(p, x["q"][0, 0], x["k"][0, 0], v2, x["pos"])
+    assert np.array_equal(h2["v4"], h["v4"])
+    assert h2["sv"][3] == 2 * h["sv"][3]
+    assert np.array_equal(np.delete(h2["sv"], 3), np.delete(h["sv"], 3))
+
+
 def test_k_mean_and_colsum(orc):
     wl, p, x, h = _head(orc, "small")
     mean = h["k_rot"].astype(np.float64).mean(axis=0)

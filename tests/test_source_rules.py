@@ -53,3 +53,85 @@ def test_mbarrier_spins_are_bounded():
         for m in re.finditer(r"while\s*\(([^;{]*mbar_(?:try|test)_wait[^;{]*)\)", code):
             cond = m.group(1)
             assert "kSpinLimit" in cond or "Limit" in cond, (name, cond)
+
+
+_COLLECTIVE = re.compile(r"__(?:shfl(?:_xor|_up|_down)?|any|all|ballot)_sync\s*\(")
+
+
+def _blank_calls(code):
+    """The code with the argument lists of every full-mask warp collective
+    replaced by a placeholder, so that only the context of each call is left."""
+    out = []
+    i = 0
+    for m in _COLLECTIVE.finditer(code):
+        if m.start() < i:
+            continue
+        out.append(code[i:m.start()])
+        depth = 0
+        j = m.end() - 1
+        while True:
+            depth += code[j] == "("
+            depth -= code[j] == ")"
+            j += 1
+            if depth == 0:
+                break
+        out.append("WARP_COLLECTIVE")
+        i = j
+    out.append(code[i:])
+    return "".join(out)
+
+
+def _statements(code):
+    return re.split(r"[;{}]", code)
+
+
+def test_warp_collectives_are_not_conditional_operands():
+    """A full-mask shuffle or vote must be reached by every lane of the warp.
+    Written as an operand of ?:, && or ||, it is skipped by the lanes whose
+    condition short-circuits, and the lanes that reach it wait for them for
+    ever (the hang of the quantise kernel whose 'mq == 0 ? 0 : shfl' skipped
+    the shuffle on lanes of zero rows and of tokens past N).  Collectives are
+    evaluated into a value first and combined afterwards."""
+    for name, text in _sources().items():
+        for st in _statements(_blank_calls(_code(text))):
+            if "WARP_COLLECTIVE" not in st:
+                continue
+            assert "?" not in st and "&&" not in st and "||" not in st, (name, st.strip())
+
+
+def test_warp_collectives_are_not_under_per_lane_branches():
+    """No full-mask collective sits inside an if/else whose condition depends on
+    the lane or on a per-row validity flag."""
+    per_lane = re.compile(r"\b(lane|threadIdx|row_ok|valid|nvalid|in_range)\b")
+    for name, text in _sources().items():
+        code = _blank_calls(_code(text))
+        for m in re.finditer("WARP_COLLECTIVE", code):
+            # walk outwards through the enclosing braces and check each opener
+            depth = 0
+            i = m.start()
+            while i > 0:
+                i -= 1
+                c = code[i]
+                if c == "}":
+                    depth += 1
+                elif c == "{":
+                    if depth == 0:
+                        head = code[max(0, i - 300):i]
+                        head = head[max(head.rfind(";"), head.rfind("}"), head.rfind("{")) + 1:]
+                        if re.match(r"\s*(?:else\s+)?if\s*\(", head):
+                            assert not per_lane.search(head), (name, head.strip())
+                    else:
+                        depth -= 1
+
+
+def test_collective_rule_flags_the_conditional_shuffle():
+    """The checker itself: the statement that hung the quantise kernel is
+    flagged, and its corrected form (shuffle first, select after) is not."""
+    bad = "const float iq = mq == 0.0f ? 0.0f : __shfl_sync(0xFFFFFFFFu, rcp7, lane & ~1);"
+    good = ("const float sh = __shfl_sync(0xFFFFFFFFu, rcp7, lane & ~1);\n"
+            "const float iq = mq == 0.0f ? 0.0f : sh;")
+    flagged = lambda src: any("WARP_COLLECTIVE" in st and ("?" in st or "&&" in st or "||" in st)  # noqa: E731
+                              for st in _statements(_blank_calls(src)))
+    assert flagged(bad)
+    assert not flagged(good)
+    assert flagged("if (reset || __any_sync(0xFFFFFFFFu, change)) {")
