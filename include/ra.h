@@ -73,8 +73,10 @@ typedef enum { RA_DT_F32 = 0, RA_DT_BF16 = 1 } ra_dtype;
  *   block_k      keys per softmax block: 16, 32, 64 or 128.  It is part of the
  *                method: the running row maximum that the P codes use is
  *                updated once per block_k keys, and the V column sums are
- *                per block_k keys.  ra_attn_int4 implements 16, 32 and 64
- *                and returns RA_ERR_UNSUPPORTED for 128.
+ *                per block_k keys.  ra_attn_int4 implements all four; 128
+ *                runs on a pair of SMs per 256-row query tile (a cluster of
+ *                two CTAs sharing one MMA), the others on one SM per two
+ *                128-row tiles.
  */
 typedef struct {
   int B, H, N, D;
@@ -149,8 +151,10 @@ ra_status ra_attn_int4(const ra_problem* p,
  *   acc_dump  [128, ceil(N/block_k), D] int32  per-block P.V accumulator
  *             sum_j (c_ij + 8) v4[j, d]  (= sum_j c_ij v4[j,d] + 8 colsum)
  * Rows past N in the tile are left unwritten.  Dump pointers may be NULL.
- * The dump variant keeps the same arithmetic as ra_attn_int4 but folds the
- * integer accumulator into the output after every block.
+ * For block_k = 128 the dump variant only adds reads and stores: its out and
+ * lse equal those of ra_attn_int4 bit for bit.  For smaller blocks it folds
+ * the integer accumulator into the output after every block (the same values
+ * up to fp32 rounding order).
  */
 ra_status ra_test_int4_codes(const ra_problem* p,
                              const uint8_t* q4, const float* sq,
@@ -176,8 +180,8 @@ ra_status ra_test_int4_codes(const ra_problem* p,
  *           RA_L_FP32       denominator = fp32 sum of exp(S - m_c), m_c the
  *                           maximum the codes are taken against.
  * opts == NULL selects the defaults.  A mode other than the defaults is
- * implemented for block_k = 64 only (RA_ERR_UNSUPPORTED otherwise); an out of
- * range mode is RA_ERR_INVALID_ARG.  All other arguments as ra_attn_int4 /
+ * implemented for block_k = 64 and 128 (RA_ERR_UNSUPPORTED otherwise); an out
+ * of range mode is RA_ERR_INVALID_ARG.  All other arguments as ra_attn_int4 /
  * ra_test_int4_codes; in the test entry p_dump holds the stored codes (c in
  * [-8, 7], or [0, 7] for RA_P_SYMMETRIC) and acc_dump the accumulator
  * sum_j (c_ij + zero point) v4[j, d].
@@ -239,6 +243,9 @@ ra_status ra_attn_bf16_fallback(const ra_problem* p, const void* q, const void* 
  *     B*H*ceil(N/256) <= ~21000 at D = 128).
  *   - The first call on a device looks up the array's device address, with
  *     that device current; make that first call before any stream capture.
+ *     The address is kept per device together with the CUDA context it was
+ *     found in; after a device reset (a new primary context) the next call
+ *     looks it up again.
  *   - All calls on a device share the one array: calls whose work may overlap
  *     on the GPU (different streams without ordering between them) race on it.
  *     Calls ordered on one stream are safe; the array keeps the last call's

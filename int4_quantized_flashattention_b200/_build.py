@@ -15,7 +15,8 @@ COMMON = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relax
           "-I", os.path.join(os.path.dirname(PKG), "include")]
 # The prologue decides INT4 codes in fp32: no multiply-add contraction there.
 PER_FILE = {"ra_prologue.cu": ["-fmad=false"]}
-SOURCES = ["ra_host.cu", "ra_prologue.cu", "ra_attn_int4.cu", "ra_attn_bf16.cu", "ra_noalloc.cu"]
+SOURCES = ["ra_host.cu", "ra_prologue.cu", "ra_attn_int4.cu", "ra_attn_int4_pair.cu", "ra_attn_bf16.cu",
+           "ra_noalloc.cu"]
 
 
 def _newer(target: str, deps) -> bool:

@@ -769,6 +769,8 @@ cudaError_t launch_attn_int4(const ra_problem& p, const uint8_t* q4, const float
     prm.dump_s = dump->s; prm.dump_p = dump->p; prm.dump_acc = dump->acc;
   }
   *unsupported = 0;
+  if (p.block_k == 128)
+    return launch_attn_int4_pair(p, q4, sq, k4, sk, v4, sv, out, lse, dump, mode, st, unsupported);
 #define RA_CASE(DD, BB, MM)                                                                          \
   if (p.D == DD && p.block_k == BB && mode == MM)                                                    \
     return dmp ? launch_cfg<DD, BB, true, MM>(p, q4, k4, v4, prm, st)                                \

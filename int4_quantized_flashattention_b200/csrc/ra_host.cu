@@ -163,11 +163,11 @@ ra_status ra_attn_bf16_fallback(const ra_problem* p, const void* q, const void* 
 
 ra_status ra_sync_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return RA_ERR_CUDA;
-  uint32_t a = 0, b = 0, c = 0;
+  uint32_t a = 0, b = 0, c = 0, d = 0;
   if (ra::read_prologue_status(&a) != cudaSuccess || ra::read_attn_int4_status(&b) != cudaSuccess ||
-      ra::read_attn_bf16_status(&c) != cudaSuccess)
+      ra::read_attn_bf16_status(&c) != cudaSuccess || ra::read_attn_pair_status(&d) != cudaSuccess)
     return RA_ERR_CUDA;
-  const uint32_t s = a | b | c;
+  const uint32_t s = a | b | c | d;
   if (s & 2u) return RA_ERR_TIMEOUT;
   if (s & 1u) return RA_ERR_INVALID_ARG;
   return RA_OK;

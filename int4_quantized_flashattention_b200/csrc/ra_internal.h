@@ -38,6 +38,12 @@ cudaError_t launch_attn_int4(const ra_problem& p, const uint8_t* q4, const float
                              const float* sk, const uint8_t* v4, const float* sv, void* out, float* lse,
                              const AttnDump* dump, int mode, cudaStream_t st, int* unsupported);
 cudaError_t read_attn_int4_status(uint32_t* out);
+// block_k = 128: the CTA-pair kernel (ra_attn_int4_pair.cu).
+cudaError_t launch_attn_int4_pair(const ra_problem& p, const uint8_t* q4, const float* sq, const uint8_t* k4,
+                                  const float* sk, const uint8_t* v4, const float* sv, void* out, float* lse,
+                                  const AttnDump* dump, int mode, cudaStream_t st, int* unsupported);
+cudaError_t read_attn_pair_status(uint32_t* out);
+cudaError_t read_attn_pair_diag(uint32_t* out);
 cudaError_t read_attn_int4_diag(uint32_t* out);  // first timed-out wait site (diagnosis)
 
 cudaError_t launch_attn_bf16(const ra_problem& p, const void* q, const void* k, const void* v, void* out,

@@ -21,23 +21,53 @@ constexpr size_t kScratchBytes = RA_STATIC_SCRATCH_BYTES;
 // device address is obtained with cudaGetSymbolAddress below.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
+// Looked-up addresses, one per device, each with the context it belongs to:
+// a device reset (or any other teardown of the primary context) reloads the
+// library's device code, and the array may then live at another address, so
+// an entry is only used while its context is the current one.
 constexpr int kMaxDevices = 256;
+struct Entry {
+  void* ctx = nullptr;
+  void* addr = nullptr;
+};
 std::mutex g_mutex;
-void* g_scratch_addr[kMaxDevices] = {};
+Entry g_entries[kMaxDevices];
 
-// Device address of the scratch array on the current device, looked up once per
-// device (the first call on a device does it, with that device current).
+// The current context of the calling thread (driver entry point, fetched once).
+void* current_context() {
+  using Fn = int (*)(void**);
+  static Fn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<Fn>(p);
+  }
+  void* ctx = nullptr;
+  if (fn == nullptr || fn(&ctx) != 0) return nullptr;
+  return ctx;
+}
+
+// Device address of the scratch array on the current device and context,
+// looked up with that device current on the first call in a context.
 ra_status scratch_address(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return RA_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return RA_ERR_UNSUPPORTED;
+  void* ctx = current_context();   // NULL before the runtime has made a context current
   std::lock_guard<std::mutex> lock(g_mutex);
-  if (g_scratch_addr[dev] == nullptr) {
+  Entry& e = g_entries[dev];
+  if (ctx == nullptr || e.addr == nullptr || e.ctx != ctx) {
+    // The lookup itself makes the device's primary context current if needed.
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return RA_ERR_CUDA;
-    g_scratch_addr[dev] = p;
+    e.addr = p;
+    e.ctx = current_context();
   }
-  *out = g_scratch_addr[dev];
+  *out = e.addr;
   return RA_OK;
 }
 

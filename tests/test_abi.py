@@ -105,15 +105,22 @@ def test_workspace_too_small_rejected(ra):
     assert rc == 1   # unknown input dtype
 
 
-def test_block_k_128_is_reported_unsupported(ra):
+def test_block_k_128_is_dispatched(ra):
+    """block_k = 128 (the CTA-pair kernel) passes validation and is not
+    refused as unsupported, in every mode; without a GPU the launch itself
+    then fails with RA_ERR_CUDA."""
     p = _wan(ra, block_k=128)
     good = C.c_void_p(0x10000)
-    assert ra.lib().ra_attn_int4(C.byref(p), *([good] * 7), None, None) == 2
+    L = ra.lib()
+    assert L.ra_attn_int4(C.byref(p), *([good] * 7), None, None) not in (1, 2)
+    for pm, lm in ((1, 0), (2, 0), (0, 1), (1, 1), (2, 1)):
+        opts = ra.AttnOpts(pm, lm)
+        assert L.ra_attn_int4_opts(C.byref(p), C.byref(opts), *([good] * 7), None, None) not in (1, 2)
 
 
 def test_ablation_options_are_validated_before_any_launch(ra):
     """Out-of-range switches are invalid; switches other than the defaults are
-    implemented for block_k = 64 only."""
+    implemented for block_k = 64 and 128 only."""
     good = C.c_void_p(0x10000)
     L = ra.lib()
     p = _wan(ra)

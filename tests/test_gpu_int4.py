@@ -174,6 +174,13 @@ def test_small_workloads_end_to_end(ra, dev, orc, name):
     (128, (44, 42, 42), 64, 3, (2, 10, 10)),    # full Hadamard rotation, N = 200
     (128, (16, 56, 56), 16, 3, (2, 5, 9)),      # full rotation, N = 90, block_k 16
     (64, (24, 20, 20), 32, 3, (5, 9, 11)),      # full rotation, D = 64
+    # block_k = 128: the CTA-pair kernel (256-row query tiles)
+    (128, (44, 42, 42), 128, 1, (2, 10, 10)),   # N = 200: one ragged key block, half-empty pair tile
+    (128, (16, 56, 56), 128, 2, (3, 7, 13)),    # N = 273: two tiles of the pair, ragged
+    (64, (24, 20, 20), 128, 1, (5, 9, 11)),     # N = 495, D = 64
+    (128, (44, 42, 42), 128, 2, (1, 1, 1)),     # N = 1
+    (128, (44, 42, 42), 128, 3, (4, 11, 13)),   # N = 572, full rotation, odd CTA of the last pair empty
+    (64, (24, 20, 20), 128, 0, (1, 1, 7)),      # N = 7, no rotation
 ])
 def test_shapes_and_ragged_tails(ra, dev, orc, D, seg, bk, rot, grid):
     wl = si.WORKLOADS["small"].with_(name=f"case{D}_{bk}", D=D, seg=seg, block_k=bk, rot=rot, grid=grid, H=3)
@@ -295,6 +302,8 @@ def test_repeat_runs_are_bitwise_identical(ra, dev):
 @pytest.mark.parametrize("p_mode,l_mode", [(0, 1), (1, 0), (1, 1), (2, 0), (2, 1)])
 @pytest.mark.parametrize("name,shape", [
     ("small", None),
+    ("small", dict(D=128, seg=(44, 42, 42), block_k=128, grid=(3, 10, 10), H=2)),  # pair kernel, N = 300
+    ("small", dict(D=64, seg=(24, 20, 20), block_k=128, grid=(5, 9, 11), H=2)),    # pair kernel, D = 64
     ("small", dict(D=128, seg=(44, 42, 42), block_k=64, grid=(2, 10, 10), H=2)),   # N = 200, ragged
     ("small", dict(D=64, seg=(24, 20, 20), block_k=64, grid=(5, 9, 11), H=2)),     # D = 64, N = 495
 ])
@@ -303,7 +312,8 @@ def test_ablation_switches(ra, dev, orc, p_mode, l_mode, name, shape):
     alternatives of key design 2) against the oracle's switches: S_int and the
     accumulators bit-exact, codes within the exponential's tie window, O within
     1e-3 on the kernel's own codes and end to end."""
-    wl = si.WORKLOADS[name] if shape is None else si.WORKLOADS[name].with_(name=f"abl_{shape['D']}", **shape)
+    wl = si.WORKLOADS[name] if shape is None else si.WORKLOADS[name].with_(
+        name=f"abl_{shape['D']}_{shape['block_k']}", **shape)
     x = si.make_inputs(wl)
     p, codes, host = gu.gpu_forward(ra, wl, x, dev, with_lse=True, p_mode=p_mode, l_mode=l_mode)
     tc = TileCheck(ra, orc, wl, p, codes, host, p_mode=p_mode, l_mode=l_mode)
@@ -347,3 +357,23 @@ def test_batch_of_two(ra, dev, orc):
     R = min(128, wl.N)
     ref = orc.attention_int4_rows(po, hc, 0, R, dumps=True)
     assert np.array_equal(s.cpu().numpy()[:R], ref["s_int"])
+
+
+@pytest.mark.parametrize("D,seg,grid", [
+    (128, (44, 42, 42), (4, 11, 13)),   # N = 572
+    (64, (24, 20, 20), (5, 9, 11)),     # N = 495
+])
+@pytest.mark.parametrize("p_mode,l_mode", [(0, 0), (1, 1), (2, 0)])
+def test_dump_variant_matches_production_bitwise(ra, dev, orc, D, seg, grid, p_mode, l_mode):
+    """The test entry (block_k = 128) runs the kernel with the dumps switched on
+    but the same arithmetic and fold schedule: its out and lse equal those of
+    ra_attn_int4 bit for bit, for the dumped tile and every other row."""
+    import torch
+    wl = si.WORKLOADS["small"].with_(name=f"dumpid{D}", D=D, seg=seg, grid=grid, block_k=128, H=2, rot=1)
+    x = si.make_inputs(wl)
+    p, codes, host = gu.gpu_forward(ra, wl, x, dev, with_lse=True, p_mode=p_mode, l_mode=l_mode)
+    for h, tile in ((0, 0), (1, 3), (1, 1)):
+        out, lse, _, _, _ = ra.test_int4_codes(p, codes, 0, h, tile, p_mode=p_mode, l_mode=l_mode)
+        assert ra.sync_status() == 0
+        assert np.array_equal(out.float().cpu().numpy(), host["out"]), (h, tile)
+        assert np.array_equal(lse.cpu().numpy(), host["lse"]), (h, tile)

@@ -4,6 +4,8 @@
   status word, and a trapped kernel would take its context down.
 * No TMA or bulk load with cluster multicast: every load of the library may
   run in multi-GPU jobs (one process per GPU), where such loads are not used.
+  (The pair attention's tcgen05.commit multicast is a completion signal, not a
+  load, and is the one multicast form allowed.)
 * No batched memory-copy entry points of the runtime or driver.
 * Every spin on an mbarrier is bounded: the waits go through the helpers that
   carry an iteration or time limit.
@@ -36,8 +38,14 @@ def test_no_device_trap_or_assert():
 
 
 def test_no_multicast_loads():
+    """The only cluster-multicast form in the library is the tcgen05.commit
+    completion signal of the CTA-pair attention (an mbarrier arrive in both
+    CTAs); no TMA or bulk copy names multicast."""
     for name, text in _sources().items():
-        assert ".multicast::cluster" not in _code(text), name
+        for line in _code(text).splitlines():
+            if ".multicast::cluster" in line:
+                assert "tcgen05.commit" in line and "cp.async" not in line, (name, line.strip())
+        assert not re.search(r"cp\.async\.bulk[^;]*multicast", _code(text)), name
 
 
 def test_no_batched_copies():
@@ -99,12 +107,25 @@ def test_warp_collectives_are_not_conditional_operands():
             assert "?" not in st and "&&" not in st and "||" not in st, (name, st.strip())
 
 
+_TMEM_COLLECTIVE = re.compile(r"\btmem_(?:ld|st)_h\d*\s*(?:<[^>]*>)?\s*\(")
+
+
+def _blank_tmem_calls(code):
+    """The code with every warp-collective tensor-memory load / store helper
+    call (tcgen05.ld / tcgen05.st .sync.aligned) replaced by the placeholder."""
+    return _TMEM_COLLECTIVE.sub("WARP_COLLECTIVE(", code)
+
+
 def test_warp_collectives_are_not_under_per_lane_branches():
-    """No full-mask collective sits inside an if/else whose condition depends on
-    the lane or on a per-row validity flag."""
-    per_lane = re.compile(r"\b(lane|threadIdx|row_ok|valid|nvalid|in_range)\b")
+    """No full-mask collective -- shuffle, vote, or tensor-memory load/store
+    (tcgen05.ld / st are .sync.aligned: every lane of the warp must execute
+    them) -- sits inside an if/else whose condition depends on the lane or on a
+    per-row flag or value (validity, the dumped tile, a row's rescale factor).
+    Such branches guard only the per-lane work; the collective runs for the
+    whole warp, with a warp vote deciding whether it runs at all."""
+    per_lane = re.compile(r"\b(lane|threadIdx|row_ok|valid|nvalid|in_range|dump_tile|sc|grow|change|near_bound|write)\b")
     for name, text in _sources().items():
-        code = _blank_calls(_code(text))
+        code = _blank_calls(_blank_tmem_calls(_code(text)))
         for m in re.finditer("WARP_COLLECTIVE", code):
             # walk outwards through the enclosing braces and check each opener
             depth = 0
@@ -135,3 +156,25 @@ def test_collective_rule_flags_the_conditional_shuffle():
     assert flagged(bad)
     assert not flagged(good)
     assert flagged("if (reset || __any_sync(0xFFFFFFFFu, change)) {")
+
+
+def test_collective_rule_flags_tensor_memory_access_under_a_row_condition():
+    """The checker flags a tensor-memory load guarded by a per-row value (the
+    rescale of one row's output accumulator), and accepts the warp-voted form."""
+    bad = ("if (sc != 1.0f) {\n  uint32_t f[32];\n  tmem_ld_h<32, kHD>(tF + c, f);\n}\n")
+    good = ("const bool any_rescale = __any_sync(0xFFFFFFFFu, sc != 1.0f);\n"
+            "if (any_rescale) {\n  uint32_t f[32];\n  tmem_ld_h<32, kHD>(tF + c, f);\n}\n")
+    per_lane = re.compile(r"\b(lane|threadIdx|row_ok|valid|nvalid|in_range|dump_tile|sc|grow|change|near_bound|write)\b")
+
+    def flagged(src):
+        code = _blank_calls(_blank_tmem_calls(src))
+        for m in re.finditer("WARP_COLLECTIVE", code):
+            head = code[:m.start()]
+            i = head.rfind("{")
+            opener = head[:i]
+            opener = opener[max(opener.rfind(";"), opener.rfind("}"), opener.rfind("{")) + 1:]
+            if re.match(r"\s*(?:else\s+)?if\s*\(", opener) and per_lane.search(opener):
+                return True
+        return False
+    assert flagged(bad)
+    assert not flagged(good)

@@ -50,6 +50,7 @@ def test_noalloc_matches_workspace_entry_on_two_calls(ra):
     ref = {n: t.clone() for n, t in ra.rope_rotate_quant(p, q, k, v, pos).items()}
     assert ra.sync_status() == 0
     fn = _c_entry(ra)
+    free_after = []
     for call in range(2):
         out = {n: torch.full_like(t, 0x5A if t.dtype == torch.uint8 else 7) for n, t in ref.items()}
         ptr = lambda t: C.c_void_p(t.data_ptr())  # noqa: E731
@@ -59,6 +60,8 @@ def test_noalloc_matches_workspace_entry_on_two_calls(ra):
                 C.c_void_p(torch.cuda.current_stream().cuda_stream))
         assert rc == 0, call
         assert ra.sync_status() == 0
+        torch.cuda.synchronize()
+        free_after.append(torch.cuda.mem_get_info()[0])
         for n in ref:
             a, b = out[n].cpu().numpy(), ref[n].cpu().numpy()
             if n in ("q4", "k4", "v4"):
@@ -69,3 +72,17 @@ def test_noalloc_matches_workspace_entry_on_two_calls(ra):
                 assert np.array_equal(a, b), (call, n)
             else:
                 assert np.allclose(a, b, rtol=1e-6, atol=0), (call, n)
+    # The point of the entry: once the first call has looked up the array (and
+    # the kernels are loaded), a call takes no device memory.
+    assert free_after[1] == free_after[0], free_after
+
+
+def test_noalloc_source_calls_no_allocator():
+    """The allocation-free entry's source names no device allocator or free
+    (host check, no GPU needed)."""
+    import os
+    import re
+    path = os.path.join(os.path.dirname(__file__), "..", "int4_quantized_flashattention_b200", "csrc", "ra_noalloc.cu")
+    code = re.sub(r"//[^\n]*", "", open(path).read())
+    for name in ("cudaMalloc", "cudaFree", "cuMemAlloc", "cuMemFree", "cudaMallocAsync", "cudaMallocManaged"):
+        assert name not in code, name
