@@ -247,6 +247,36 @@ __device__ __forceinline__ bool pwait(uint64_t* bar, uint32_t parity, const Abor
   return r > 0;
 }
 
+// As pwait, for all 32 lanes of a warp together: the lanes test the barrier
+// and decide as one (warp votes), so the warp stays converged through the wait
+// and the warp-collective tensor-memory accesses after it.
+__device__ __forceinline__ bool pwait_warp(uint64_t* bar, uint32_t parity, const Abort& ab, uint32_t site, uint32_t g,
+                                           uint32_t rank, uint32_t backoff_ns = 32) {
+  const bool first = mbar_test_wait(bar, parity);
+  if (__all_sync(0xFFFFFFFFu, first)) return true;
+  const uint64_t t0 = global_ns();
+  uint32_t sleep = 16;
+  for (uint32_t n = 1;; ++n) {
+    __nanosleep(sleep);
+    const bool done = mbar_test_wait(bar, parity);
+    if (__all_sync(0xFFFFFFFFu, done)) return true;
+    sleep = min(sleep * 2, backoff_ns);
+    if ((n & 31u) == 0) {
+      const bool aborted = *ab.local != 0;
+      const bool late = global_ns() - t0 > kWaitLimitNs;
+      const bool any_aborted = __any_sync(0xFFFFFFFFu, aborted);
+      const bool any_late = __any_sync(0xFFFFFFFFu, late);
+      if (any_late && !any_aborted) {
+        if ((threadIdx.x & 31) == 0) {
+          ab.raise();
+          note_timeout_p(site, g, rank);
+        }
+      }
+      if (any_aborted || any_late) return false;
+    }
+  }
+}
+
 // MODE bits 0-1: P codes (0 range-rectified, 1 block-local maximum, 2
 // symmetric); bit 2: fp32 denominator.
 template <int D, bool DUMP, int MODE>
@@ -437,8 +467,8 @@ attn_int4_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             return key < prm.N ? __ldg(skh + key) * (1.0f / 256.0f) : __int_as_float(0x7FC00000);
           };
           float sc0 = load_sc(0, wt), sc1 = load_sc(0, wt + 64);
-          if (!(ok = pwait(B.qpk_full, li & 1, ab, 8u, li, rank, 256u))) break;
-          if (!(ok = pwait(B.q_free, (li & 1) ^ 1, ab, 9u, li, rank, 256u))) break;
+          if (!(ok = pwait_warp(B.qpk_full, li & 1, ab, 8u, li, rank, 256u))) break;
+          if (!(ok = pwait_warp(B.q_free, (li & 1) ^ 1, ab, 9u, li, rank, 256u))) break;
           widen_rows<kRowsP, D / 2>(smem + C::oQPk, smem + C::oQ, wt);
           fence_proxy_async_smem();
           __syncwarp();
@@ -446,20 +476,21 @@ attn_int4_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           for (int t = 0; t < nb; ++t, ++g) {
             const int s = g % S;
             const uint32_t ph = ((g / S) & 1) ^ 1;
-            // the next block's scales, in flight while this block is widened
-            const float nx0 = t + 1 < nb ? load_sc(t + 1, wt) : 0.0f;
-            const float nx1 = t + 1 < nb ? load_sc(t + 1, wt + 64) : 0.0f;
-            if (!(ok = pwait(B.pk_full + s, (g / S) & 1, ab, 10u, g, rank, 128u))) break;
+            if (!(ok = pwait_warp(B.pk_full + s, (g / S) & 1, ab, 10u, g, rank, 128u))) break;
             const uint8_t* pk = smem + C::oPk + s * (C::kKPk + C::kVPk);
-            if (!(ok = pwait(B.kw_empty + s, ph, ab, 11u, g, rank, 256u))) break;
+            if (!(ok = pwait_warp(B.kw_empty + s, ph, ab, 11u, g, rank, 256u))) break;
             planK.run(pk, smem + C::oKw + s * C::kKwStride);
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) { mbar_arrive_cluster(lead(B.kw_full + s)); mbar_arrive(B.pk_empty + s); }
+            // The next block's scales, requested after the cluster-scope
+            // release above (which would otherwise wait for these loads).
+            const float nx0 = t + 1 < nb ? load_sc(t + 1, wt) : 0.0f;
+            const float nx1 = t + 1 < nb ? load_sc(t + 1, wt + 64) : 0.0f;
             // Per-key scales of the whole block (both CTAs' softmax rows use
             // all 128 keys).  Keys past N get a NaN scale: their score is NaN,
             // which the maximum ignores, and their code bytes are masked.
-            if (!(ok = pwait(B.ksc_empty + s, ph, ab, 12u, g, rank, 256u))) break;
+            if (!(ok = pwait_warp(B.ksc_empty + s, ph, ab, 12u, g, rank, 256u))) break;
             float* ksc = reinterpret_cast<float*>(smem + C::oKsc) + s * kBK;
             ksc[wt] = sc0;
             ksc[wt + 64] = sc1;
@@ -476,9 +507,9 @@ attn_int4_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           for (int t = 0; t < nb; ++t, ++g) {
             const int s = g % S;
             const uint32_t ph = ((g / S) & 1) ^ 1;
-            if (!(ok = pwait(B.pk_full + s, (g / S) & 1, ab, 10u, g, rank, 128u))) break;
+            if (!(ok = pwait_warp(B.pk_full + s, (g / S) & 1, ab, 10u, g, rank, 128u))) break;
             const uint8_t* pk = smem + C::oPk + s * (C::kKPk + C::kVPk);
-            if (!(ok = pwait(B.vw_empty + s, ph, ab, 13u, g, rank, 256u))) break;
+            if (!(ok = pwait_warp(B.vw_empty + s, ph, ab, 13u, g, rank, 256u))) break;
             planV.run(pk + C::kKPk, smem + C::oVw + s * C::kVwStride);
             fence_proxy_async_smem();
             __syncwarp();
@@ -530,18 +561,23 @@ attn_int4_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     // before the next load of these columns) covers them.
     auto fold = [&](float coef, bool reset) __attribute__((always_inline)) {
       const float2 w2 = make_float2(coef, coef);
+      uint32_t a[kHD], f[kHD];
+      // every column of this thread in one round trip (D = 64: one pair of loads)
+      if constexpr (kHD == 64) {
+        tmem_ld_h32_quad<kHD>(tA, tF, tA + 32, tF + 32, a, f, a + 32, f + 32);
+      } else {
+        tmem_ld_h32_pair<kHD>(tA, tF, a, f);
+      }
+#pragma unroll
+      for (int q = 0; q < kHD; q += 2) {
+        const float2 x = __fadd2_rn(make_float2(__uint_as_float(a[q]), __uint_as_float(a[q + 1])), kNegMagic2);
+        const float2 y = __ffma2_rn(w2, x, make_float2(__uint_as_float(f[q]), __uint_as_float(f[q + 1])));
+        f[q] = __float_as_uint(y.x);
+        f[q + 1] = __float_as_uint(y.y);
+      }
 #pragma unroll
       for (int c = 0; c < kHD; c += 32) {
-        uint32_t a[32], f[32];
-        tmem_ld_h32_pair<kHD>(tA + c, tF + c, a, f);
-#pragma unroll
-        for (int q = 0; q < 32; q += 2) {
-          const float2 x = __fadd2_rn(make_float2(__uint_as_float(a[q]), __uint_as_float(a[q + 1])), kNegMagic2);
-          const float2 y = __ffma2_rn(w2, x, make_float2(__uint_as_float(f[q]), __uint_as_float(f[q + 1])));
-          f[q] = __float_as_uint(y.x);
-          f[q + 1] = __float_as_uint(y.y);
-        }
-        tmem_st_h32_nw<kHD>(tF + c, f);
+        tmem_st_h32_nw<kHD>(tF + c, f + c);
         if (reset) tmem_fill_h32_nw<kHD>(tA + c, kMagicP);
       }
     };
@@ -568,9 +604,8 @@ attn_int4_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     // Reads S of block gs (after its Q K^T) from S buffer gs & 1; both halves
     // of the warp read 64 keys.
     auto take_s = [&](uint32_t gs, uint32_t* raw) __attribute__((always_inline)) -> bool {
-      if (!pwait(B.s_full + (gs & 1), (gs >> 1) & 1, ab, 14u, gs, rank, 16u)) return false;
-      if (!pwait(B.ksc_full + gs % S, (gs / S) & 1, ab, 15u, gs, rank, 16u)) return false;
-      __syncwarp();
+      if (!pwait_warp(B.s_full + (gs & 1), (gs >> 1) & 1, ab, 14u, gs, rank, 16u)) return false;
+      if (!pwait_warp(B.ksc_full + gs % S, (gs / S) & 1, ab, 15u, gs, rank, 16u)) return false;
       tc_fence_after();
       tmem_ld_h64<kHK>(tbase + C::tS + (gs & 1) * 128 + lane_off, raw);
       return true;
@@ -679,9 +714,10 @@ attn_int4_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         tmem_st_h16_nw<kHK / 4>(tbase + C::tS + (gg & 1) * 128 + lane_off, words);
         // Sum of the row's codes (+8 each): bytes are at most 15, so plain
         // word additions of 16 words cannot carry between bytes.
-        uint32_t wsum = 0;
+        uint32_t ws4[4] = {0u, 0u, 0u, 0u};   // four independent chains
 #pragma unroll
-        for (int q = 0; q < kHK / 4; ++q) wsum += words[q];
+        for (int q = 0; q < kHK / 4; ++q) ws4[q & 3] += words[q];
+        const uint32_t wsum = (ws4[0] + ws4[1]) + (ws4[2] + ws4[3]);
         int lq = static_cast<int>(__dp4a(wsum, 0x01010101u, 0u));
         lq += __shfl_xor_sync(0xFFFFFFFFu, lq, 16);
         float le = 0.0f;
@@ -728,8 +764,7 @@ attn_int4_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         }
         if (reset || any_change || dump_now) {
           // A holds the P.V results up to block t - 1.
-          if (!(ok = pwait(B.pv_done + ((gg - 1) & 1), ((gg - 1) >> 1) & 1, ab, 16u, gg, rank, 16u))) return;
-          __syncwarp();
+          if (!(ok = pwait_warp(B.pv_done + ((gg - 1) & 1), ((gg - 1) >> 1) & 1, ab, 16u, gg, rank, 16u))) return;
           tc_fence_after();
           if (DUMP && dump_now) {
             dump_acc(t - 1, r, dump_reset, dump_tile);
@@ -775,8 +810,7 @@ attn_int4_pair_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       g = g0 + nb;
       if (!ok) break;
       // Last block: fold the accumulator into F (and reset it), normalise, store.
-      if (!(ok = pwait(B.pv_done + ((g - 1) & 1), ((g - 1) >> 1) & 1, ab, 17u, g, rank, 16u))) break;
-      __syncwarp();
+      if (!(ok = pwait_warp(B.pv_done + ((g - 1) & 1), ((g - 1) >> 1) & 1, ab, 17u, g, rank, 16u))) break;
       tc_fence_after();
       if constexpr (DUMP) {
         const bool any_dump = __any_sync(0xFFFFFFFFu, dump_tile);

@@ -94,3 +94,42 @@ def test_bf16_fallback_long_sequence(ra, orc):
     """4096 keys (64 blocks): many running-maximum changes and folds."""
     wl = si.WORKLOADS["sweep4096"].with_(H=2)
     _run(ra, orc, wl, heads=(0, 1))
+
+
+def test_bf16_fallback_wan_sampled(ra, orc):
+    """The bf16 fallback at the size bench.py times it (wan: H = 40, N = 32760):
+    RoPE of three whole heads, attention on sampled query rows (first, middle
+    and ragged last tiles of three heads) against fp64 attention over all keys."""
+    import torch
+    wl = si.WORKLOADS["wan"]
+    dev = gu.device()
+    x = si.make_inputs(wl)
+    p = gu.problem_for(ra, wl)
+    q, k, v, pos = gu.to_device(x, wl, dev)
+    qr, kr = ra.rope_bf16(p, q, k, pos)
+    lse = torch.empty(wl.B, wl.H, wl.N, dtype=torch.float32, device=dev)
+    out = ra.attn_bf16_fallback(p, qr, kr, v, lse=lse)
+    assert ra.sync_status() == 0
+    po = orc.problem(wl)
+    po.rot = 0
+    num = den = 0.0
+    for h in (0, 19, 39):
+        qr_h, kr_h = qr[0, h].float().cpu().numpy(), kr[0, h].float().cpu().numpy()
+        for name, src, got in (("q", x["q"], qr_h), ("k", x["k"], kr_h)):
+            ref = gu.bf16_round(orc.rope_rotate(po, src[0, h], x["pos"]))
+            u = _bf16_ulps(got, ref)
+            assert u.max() <= 1.0, (name, h, u.max())
+            assert np.mean(u == 0) >= 0.999, (name, h)
+        v64 = v[0, h].float().cpu().numpy().astype(np.float64)
+        k64 = kr_h.astype(np.float64)
+        rows = np.concatenate([np.arange(0, 128), np.arange(16384, 16512), np.arange(wl.N - 120, wl.N)])
+        q64 = qr_h[rows].astype(np.float64)
+        ref = orc.reference_attention_fp64(q64, k64, v64)
+        s = q64 @ k64.T / math.sqrt(wl.D)
+        m = s.max(axis=1)
+        ref_lse = m + np.log(np.exp(s - m[:, None]).sum(axis=1))
+        got = out[0, h].float().cpu().numpy()[rows]
+        assert np.max(np.abs(lse[0, h].cpu().numpy()[rows] - ref_lse)) <= 2e-3, h
+        num += float(np.sum((got - ref) ** 2))
+        den += float(np.sum(ref ** 2))
+    assert math.sqrt(num / den) <= 5e-3, math.sqrt(num / den)

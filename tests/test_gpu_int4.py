@@ -250,8 +250,9 @@ def test_position_outside_grid_is_reported(ra, dev):
 # --- full-size workloads: sampled heads and query tiles ----------------------
 
 @pytest.mark.parametrize("name,heads,tiles", [
-    ("wan", (0, 23, 39), tuple((h, t) for h in (0, 7, 23, 30, 39) for t in (0, 50, 100, 128, 200, 255))),
-    ("hunyuan", (5,), ((5, 0), (5, 928), (11, 464), (17, 100))),
+    # every head's prologue outputs in full (O(N D) each), attention on sampled tiles
+    ("wan", tuple(range(40)), tuple((h, t) for h in (0, 7, 23, 30, 39) for t in (0, 50, 100, 128, 200, 255))),
+    ("hunyuan", tuple(range(24)), ((5, 0), (5, 928), (11, 464), (17, 100), (23, 928))),
 ])
 def test_full_size_sampled(ra, dev, orc, name, heads, tiles):
     wl = si.WORKLOADS[name]
@@ -377,3 +378,56 @@ def test_dump_variant_matches_production_bitwise(ra, dev, orc, D, seg, grid, p_m
         assert ra.sync_status() == 0
         assert np.array_equal(out.float().cpu().numpy(), host["out"]), (h, tile)
         assert np.array_equal(lse.cpu().numpy(), host["lse"]), (h, tile)
+
+
+@pytest.mark.parametrize("name", ["sweep8192", "sweep8192_half", "sweep16384", "sweep16384_half",
+                                  "sweep32760_half", "sweep65536", "sweep65536_half"])
+def test_sweep_sampled(ra, dev, orc, name):
+    """The sweep shapes (H = 40, D = 128) at full size in both rotation modes:
+    the prologue of two heads in full, and the first, middle and last (for
+    N = 32760 ragged) query tiles of those heads through the test entry."""
+    wl = si.WORKLOADS[name]
+    x = si.make_inputs(wl)
+    p, codes, host = gu.gpu_forward(ra, wl, x, dev, with_lse=True)
+    assert np.all(np.isfinite(host["out"])) and np.all(np.isfinite(host["lse"]))
+    _check_prologue(orc, wl, x, host, (0, 39))
+    ntiles = -(-wl.N // 128)
+    tc = TileCheck(ra, orc, wl, p, codes, host)
+    for h in (0, 39):
+        for t in (0, ntiles // 2, ntiles - 1):
+            tc.tile(h, t)
+    assert tc.end_to_end() <= 1e-3, (tc.end_to_end(), tc.flips, tc.relevant)
+
+
+def test_sharp_p_at_n16384(ra, dev, orc):
+    """The sharp-P variant (Q x 8: near one-hot softmax rows) at N = 16384."""
+    wl = si.WORKLOADS["sweep16384"].with_(sharp=True, name="sweep16384_sharp")
+    x = si.make_inputs(wl)
+    p, codes, host = gu.gpu_forward(ra, wl, x, dev, with_lse=True)
+    _check_prologue(orc, wl, x, host, (3,))
+    tc = TileCheck(ra, orc, wl, p, codes, host)
+    for h, t in ((3, 0), (3, 64), (3, 127), (21, 77)):
+        tc.tile(h, t)
+    assert tc.end_to_end() <= 1e-3, (tc.end_to_end(), tc.flips, tc.relevant)
+
+
+def test_dump_variant_for_small_blocks_matches_up_to_rounding(ra, dev, orc):
+    """For block_k <= 64 the test entry folds the integer accumulator after
+    every block instead of only when a row maximum grows: the same sums in
+    another fp32 order, so out agrees with ra_attn_int4 to fp32 rounding."""
+    wl = si.WORKLOADS["small"].with_(name="dump64", grid=(4, 11, 13), H=2)
+    x = si.make_inputs(wl)
+    p, codes, host = gu.gpu_forward(ra, wl, x, dev, with_lse=True)
+    out, lse, _, _, _ = ra.test_int4_codes(p, codes, 0, 1, 2)
+    assert ra.sync_status() == 0
+    got = out.float().cpu().numpy()
+    ref = host["out"]
+    # bf16 outputs: equal, or apart by the fp32 difference of the two summation
+    # orders carried through a bf16 rounding -- at most one bf16 unit of the
+    # row's largest magnitude (outputs near zero come from cancellation, so
+    # the bound is taken per row, not per element)
+    row_scale = np.abs(ref).max(axis=-1, keepdims=True)
+    assert np.all(np.abs(got - ref) <= row_scale * 2.0 ** -7), np.max(np.abs(got - ref) / row_scale)
+    assert gu.rel_l2(got, ref) <= 1e-4, gu.rel_l2(got, ref)
+    assert np.mean(got != ref) <= 1e-2, np.mean(got != ref)
+    assert np.allclose(lse.cpu().numpy(), host["lse"], rtol=0, atol=1e-5)
