@@ -90,9 +90,10 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(self.samples)}
 
 
-def _workload(name):
+def _workload(name, block_k=None):
     from synth import inputs as si
-    return si.WORKLOADS[name]
+    wl = si.WORKLOADS[name]
+    return wl if block_k is None else wl.with_(block_k=block_k)
 
 
 def _config(wl, extra=None):
@@ -137,6 +138,7 @@ def cpu_baseline(wl, target_s: float = 15.0, x=None):
     t = t_att + t_pro * rows / wl.N
     ops = 4.0 * rows * wl.N * wl.D
     return {"value": ops / t / 1e12, "unit": "TOPS", "cores": oracle.num_threads(), "kind": "oracle",
+            "seconds": t,
             "sample": f"head 0 of {wl.name}: prologue of all {wl.N} tokens (prorated to the rows) + "
                       f"attention of {rows} query rows over all {wl.N} keys; {t:.1f} s of CPU time"}
 
@@ -190,7 +192,7 @@ def run_ours(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    wl = _workload(args.workload)
+    wl = _workload(args.workload, args.block_k)
     x = si.make_inputs(wl)
     p = ra.Problem.make(wl.B, wl.H, wl.D, wl.seg, wl.grid, theta=wl.theta, rot=wl.rot,
                         block_q=wl.block_q, block_k=wl.block_k)
@@ -301,15 +303,18 @@ def run_ours(args, rank, world, local_rank):
     # not part of the INT4 step, reported against the bf16 tensor peak.
     qr, kr = ra.rope_bf16(p, q, k, pos, workspace=ws)
     out_b = torch.empty_like(out)
+    # the fallback's key block (a tiling choice that leaves its result unchanged)
+    pb = ra.Problem.make(wl.B, wl.H, wl.D, wl.seg, wl.grid, theta=wl.theta, rot=wl.rot,
+                         block_q=wl.block_q, block_k=min(wl.block_k, 64))
     for _ in range(2):
-        ra.attn_bf16_fallback(p, qr, kr, v, out=out_b)
+        ra.attn_bf16_fallback(pb, qr, kr, v, out=out_b)
     torch.cuda.synchronize(dev)
     fb = []
     for _ in range(max(3, args.steps // 4)):
         a0 = torch.cuda.Event(enable_timing=True)
         a1 = torch.cuda.Event(enable_timing=True)
         a0.record(stream)
-        ra.attn_bf16_fallback(p, qr, kr, v, out=out_b)
+        ra.attn_bf16_fallback(pb, qr, kr, v, out=out_b)
         a1.record(stream)
         torch.cuda.synchronize(dev)
         fb.append(a0.elapsed_time(a1))
@@ -322,7 +327,7 @@ def run_ours(args, rank, world, local_rank):
     # fp32 denominator), each timed on its own on the same codes; not part of
     # the INT4 step.
     abl = {}
-    if wl.block_k == 64:
+    if wl.block_k in (64, 128) and not args.quick:
         for name, pm, lm in ABLATIONS:
             for _ in range(2):
                 ra.attn_int4(p, codes, out=out, p_mode=pm, l_mode=lm)
@@ -343,7 +348,7 @@ def run_ours(args, rank, world, local_rank):
     # The prologue under each rotation mode (full D x D Hadamard against the
     # 2x2 rotations), timed on the same inputs after everything else.
     rot_ms = {}
-    for rname, rmode in (("interleaved", ra.ROT_INTERLEAVED), ("half", ra.ROT_HALF), ("full", ra.ROT_FULL),
+    for rname, rmode in () if args.quick else (("interleaved", ra.ROT_INTERLEAVED), ("half", ra.ROT_HALF), ("full", ra.ROT_FULL),
                          ("none", ra.ROT_NONE)):
         pr = ra.Problem.make(wl.B, wl.H, wl.D, wl.seg, wl.grid, theta=wl.theta, rot=rmode,
                              block_q=wl.block_q, block_k=wl.block_k)
@@ -383,7 +388,7 @@ def run_ours(args, rank, world, local_rank):
         "roofline": {"bound": "tensor", "kernel": "attn_int4_kernel", "achieved": round(achieved, 1),
                      "peak": round(int8_peak, 1), "unit": "TFLOP/s", "frac": round(achieved / int8_peak, 4),
                      "peak_source": f"2 x {pk['source']} bf16 burst {pk['bf16_tflops']} TFLOP/s (int8 ops/s)",
-                     "traffic": _attn_traffic() if args.workload == "wan" else None},
+                     "traffic": _attn_traffic() if (args.workload == "wan" and args.block_k is None) else None},
         "prologue": {"ms": round(pro_med, 4), "bytes": pro_bytes,
                      "achieved_gbs": round(pro_bytes / (pro_med * 1e-3) / 1e9, 1),
                      "peak_gbs": pk["hbm_gbs"], "frac": round(pro_bytes / (pro_med * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
@@ -413,8 +418,15 @@ def prologue_bytes(wl):
 
 
 def run_reference(args):
-    """The oracle as it stands, on the host cores, one bounded sample per step."""
-    wl = _workload(args.workload)
+    """The oracle as it stands, on the host cores, one bounded sample per step.
+
+    A whole step of the workload takes the oracle many minutes, so each step
+    runs a bounded sample (the prologue of head 0 and as many query tiles as
+    fit in the per-step budget, every step within the run's few minutes); the
+    line's value is that sample's rate and ms_per_step the time the whole
+    step would take at it, marked as extrapolated, with the sample's own time
+    beside it."""
+    wl = _workload(args.workload, args.block_k)
     import oracle
     oracle.lib()
     from synth import inputs as si
@@ -422,16 +434,22 @@ def run_reference(args):
     # each step is one bounded sample; the whole run stays within a few minutes
     per_step = max(1.0, min(args.ref_seconds, 180.0 / max(1, args.warmup + args.steps)))
     vals = []
+    sample_s = []
     base = None
     for i in range(args.warmup + args.steps):
         r = cpu_baseline(wl, target_s=per_step, x=x)
         if i >= args.warmup:
             vals.append(r["value"])
+            sample_s.append(r["seconds"])
             base = r
     v = statistics.median(vals)
     ms = 4.0 * wl.N * wl.N * wl.D * wl.H * wl.B / (v * 1e12) * 1e3
     return {"metric": METRIC, "value": round(v, 6), "unit": "TOPS", "n_gpus": 1, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(ms, 1), "higher_is_better": True, "scaling": "weak",
+            "warmup": args.warmup, "ms_per_step": round(ms, 1), "extrapolated": True,
+            "sample_ms_per_step": round(1e3 * statistics.median(sample_s), 1),
+            "extrapolation": f"ms_per_step = 4 N^2 D H / value: the whole step at the sampled rate; each step "
+                             f"ran a {per_step:.1f} s sample ({base['sample']})",
+            "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "int4", "data": "synthetic (seeded, outlier-structured; no model weights)",
             "config": _config(wl), "impl": "reference",
             "cpu_baseline": {"value": round(v, 6), "unit": "TOPS", "cores": base["cores"], "kind": "oracle",
@@ -446,6 +464,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="wan")
+    ap.add_argument("--block-k", type=int, default=None, help="override the workload's key block size")
+    ap.add_argument("--quick", action="store_true",
+                    help="skip the ablation modes and the per-rotation prologue timings (for config sweeps)")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the CPU oracle sample")
     ap.add_argument("--ref-seconds", type=float, default=10.0, help="CPU seconds per reference sample")
     args = ap.parse_args()
@@ -467,7 +488,7 @@ def main():
         res = run_ours(args, rank, world, local_rank)
         if rank == 0:
             if world == 1 and not args.no_cpu_baseline:
-                res["cpu_baseline"] = cpu_baseline(_workload(args.workload))
+                res["cpu_baseline"] = cpu_baseline(_workload(args.workload, args.block_k))
             print(json.dumps(res), flush=True)
     finally:
         if world > 1:

@@ -11,7 +11,7 @@
 namespace ra {
 
 struct WorkspaceLayout {
-  size_t tab, ksum, vmax, vinv, total;
+  size_t tab, tab0, ksum, vmax, vinv, total;
 };
 
 size_t rope_table_len(const ra_problem& p);

@@ -261,26 +261,37 @@ __device__ __forceinline__ void rope_apply8(const SegInfo& s, const RopePlan& rp
 }
 
 
-// For two elements: the bits of 1.5 * 2^23 + clamp(rint(x * inv), -7, 7).
-// Clamping before rounding gives the same integer (rint is monotone and +-7
-// are integers); the code is the value minus 0x4B400000, and its low 4 bits
-// are the two's complement nibble.  f32x2 arithmetic rounds each lane exactly
-// like the scalar operations.
+// For two elements: the bits of 1.5 * 2^23 + 8 + rint(x * inv), i.e.
+// 0x4B400000 + (code + 8) with code + 8 in [1, 15].  One f32x2 fused
+// multiply-add: the product x * inv is exact inside the FMA and the single
+// rounding to the integer grid of [2^23, 2^24) (ties to even; the offset is
+// even) is the rint of the exact product.
+//   * No clamp is needed: inv = fl(7/amax) with |x| <= amax (the token's or
+//     channel's own maximum), so |x * inv| <= 7 (1 + 2^-23) < 7.5 and rint
+//     already lies in [-7, 7]; amax = 0 gives inv = 0 and code 0.
+//   * The exact product is the decision on purpose: an f32x2 multiply and an
+//     f32x2 add in sequence are fused by the compiler even when written with
+//     explicit round-to-nearest (measured: the codes of exact fp32 ties
+//     x * inv = k + 1/2 followed the unrounded product), so a two-rounding
+//     decision would need scalar operations at twice the instruction count.
+constexpr uint32_t kQBits = 0x4B400000u;       // bits of 1.5 * 2^23
+constexpr float kQMagic8 = 12582920.0f;        // 1.5 * 2^23 + 8
 __device__ __forceinline__ void quant4_bits2(float x0, float x1, float inv0, float inv1, uint32_t* b) {
-  float2 y = __fmul2_rn(make_float2(x0, x1), make_float2(inv0, inv1));
-  y.x = fminf(fmaxf(y.x, -7.0f), 7.0f);
-  y.y = fminf(fmaxf(y.y, -7.0f), 7.0f);
-  const float2 t = __fadd2_rn(y, make_float2(12582912.0f, 12582912.0f));
+  const float2 t = __ffma2_rn(make_float2(x0, x1), make_float2(inv0, inv1), make_float2(kQMagic8, kQMagic8));
   b[0] = __float_as_uint(t.x);
   b[1] = __float_as_uint(t.y);
 }
 
-// Packs the nibbles of eight quant4_bits2 results, element 2t in the low nibble.
+// Packs the nibbles of eight quant4_bits2 results, element 2t in the low
+// nibble: sum_i 16^i b_i (integer multiply-adds) minus the known sum of the
+// 0x4B400000 parts leaves the nibbles code + 8 (at most 15: no carries);
+// XOR with 8 in every nibble turns code + 8 into the two's complement code.
+constexpr uint32_t kQBitsRep = kQBits * 0x11111111u;   // sum_i 16^i 0x4B400000 mod 2^32
 __device__ __forceinline__ uint32_t pack8_bits(const uint32_t* b) {
-  uint32_t p[4];
+  uint32_t acc = b[7];
 #pragma unroll
-  for (int j = 0; j < 4; ++j) p[j] = (b[2 * j] & 0x0Fu) | ((b[2 * j + 1] << 4) & ~0x0Fu);  // byte 0 is the pair
-  return __byte_perm(__byte_perm(p[0], p[1], 0x0040), __byte_perm(p[2], p[3], 0x0040), 0x5410);
+  for (int i = 6; i >= 0; --i) acc = acc * 16u + b[i];
+  return (acc - kQBitsRep) ^ 0x88888888u;
 }
 
 // Max over the D/8 threads of a token (a contiguous lane group of size lpt).
@@ -295,7 +306,8 @@ struct PrologueArgs {
   int bk_log2;  // block_k = 2^bk_log2
   const void *q, *k, *v;
   const int32_t* pos;
-  const float2* tab;   // RoPE table entries (a, b)
+  const float2* tab;   // RoPE table entries (a, b) of the rotation mode
+  const float2* tab0;  // plain RoPE table (cos, sin): the reduce pass
   double* ksum;     // [BH, nchunk, D]
   float* vmax;      // [BH, nchunk, D]
   float* vinv;      // [BH, D]
@@ -368,14 +380,14 @@ __device__ __forceinline__ bool stage_wait(uint64_t* bar, uint32_t parity, volat
   return !__syncthreads_or(r <= 0);
 }
 
-// Pass 1: per chunk of tokens, fp64 channel sums of the rotated K and channel
-// maxima of |V|.  kRot: the rotation mode (a template parameter, so every
-// mode keeps only its own per-thread state).
-template <bool kBf16, int kRot, int kD>
+// Pass 1: per chunk of tokens, fp64 channel sums of the RoPE'd K (before the
+// rotation, which is linear and the same for every token: the finalize pass
+// applies it to the mean) and channel maxima of |V|.
+template <bool kBf16, int kD>
 __global__ void __launch_bounds__(kThreads, 3) prologue_reduce_kernel(PrologueArgs a) {
   using IO = StageIO<kBf16, 2, kStgR>;
-  // Row buffer of the half rotation's exchange (one token row per warp slot).
-  __shared__ float rows[kRot == 2 ? kThreads / 32 : 1][4][128];
+  constexpr int kRot = 0;
+  __shared__ float rows[1][4][128];   // (unused by the plain RoPE)
   __shared__ uint64_t full[kStgR];
   __shared__ int abort_flag;
   extern __shared__ __align__(128) uint8_t stg[];
@@ -383,7 +395,7 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_reduce_kernel(PrologueAr
   const int lpt = kD >> 3, tpw = 32 / lpt;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tok_in_warp = lane / lpt, c0 = (lane % lpt) * 8;
-  float* const row = rows[kRot == 2 ? warp : 0][kRot == 2 ? tok_in_warp : 0];
+  float* const row = rows[0][0];
   const int step = (kThreads / 32) * tpw;
   const int n0 = chunk * kChunk;
   const size_t head = static_cast<size_t>(bh) * a.N * kD;
@@ -425,8 +437,7 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_reduce_kernel(PrologueAr
 #pragma unroll
         for (int i = 0; i < 8; ++i) { x[i] = 0.0f; y[i] = 0.0f; }
       }
-      // Every lane takes part (the half rotation synchronises the warp).
-      rope_coef8p(a.s, rp, a.tab, gp, ca, cb);
+      rope_coef8p(a.s, rp, a.tab0, gp, ca, cb);
       rope_apply8(a.s, rp, kRot, ca, cb, c0, x, row);
       if (valid) {
 #pragma unroll
@@ -464,37 +475,61 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_reduce_kernel(PrologueAr
   }
 }
 
-// Per head and channel: K mean (fp64 sum over chunks in order, rounded once),
-// V scale amax/7 and reciprocal 7/amax.
+// Per head and channel: K mean (fp64 sum over chunks in order; the rotation
+// applied to the mean in fp64; rounded once), V scale amax/7 and reciprocal
+// 7/amax.  One CTA of 128 threads per head; threads d >= D only take part in
+// the barrier.
 __global__ void prologue_finalize_kernel(PrologueArgs a) {
+  __shared__ double m[128];
   const int bh = blockIdx.x, d = threadIdx.x;
-  if (d >= a.D) return;
-  double sum = 0.0;
-  float mx = 0.0f;
-  const size_t o0 = static_cast<size_t>(bh) * a.nchunk * a.D + d;
-  int c = 0;
-  // Eight chunks' loads in flight at a time; the sum keeps the chunk order.
-  for (; c + 8 <= a.nchunk; c += 8) {
-    double s8[8];
-    float m8[8];
+  const bool active = d < a.D;
+  if (active) {
+    double sum = 0.0;
+    float mx = 0.0f;
+    const size_t o0 = static_cast<size_t>(bh) * a.nchunk * a.D + d;
+    int c = 0;
+    // Eight chunks' loads in flight at a time; the sum keeps the chunk order.
+    for (; c + 8 <= a.nchunk; c += 8) {
+      double s8[8];
+      float m8[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      s8[u] = a.ksum[o0 + static_cast<size_t>(c + u) * a.D];
-      m8[u] = a.vmax[o0 + static_cast<size_t>(c + u) * a.D];
-    }
+      for (int u = 0; u < 8; ++u) {
+        s8[u] = a.ksum[o0 + static_cast<size_t>(c + u) * a.D];
+        m8[u] = a.vmax[o0 + static_cast<size_t>(c + u) * a.D];
+      }
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      sum += s8[u];
-      mx = fmaxf(mx, m8[u]);
+      for (int u = 0; u < 8; ++u) {
+        sum += s8[u];
+        mx = fmaxf(mx, m8[u]);
+      }
     }
+    for (; c < a.nchunk; ++c) {
+      sum += a.ksum[o0 + static_cast<size_t>(c) * a.D];
+      mx = fmaxf(mx, a.vmax[o0 + static_cast<size_t>(c) * a.D]);
+    }
+    a.sv[bh * a.D + d] = __fdiv_rn(mx, 7.0f);
+    a.vinv[bh * a.D + d] = mx == 0.0f ? 0.0f : __fdiv_rn(7.0f, mx);
+    m[d] = sum / static_cast<double>(a.N);   // mean of the RoPE'd K (before the rotation)
   }
-  for (; c < a.nchunk; ++c) {
-    sum += a.ksum[o0 + static_cast<size_t>(c) * a.D];
-    mx = fmaxf(mx, a.vmax[o0 + static_cast<size_t>(c) * a.D]);
+  __syncthreads();
+  if (!active) return;
+  const double r2 = 0.70710678118654752440;   // 1/sqrt(2) in fp64
+  double mu;
+  if (a.rot == 1) {
+    const int e = d & ~1;
+    mu = (d & 1) ? (m[e] - m[e + 1]) * r2 : (m[e] + m[e + 1]) * r2;
+  } else if (a.rot == 2) {
+    const int j = seg_of(a.s, d);
+    const int o = a.s.off[j], h = a.s.dj[j] >> 1, i = (d - o) >> 1;
+    mu = ((d - o) & 1) ? (m[o + i] - m[o + i + h]) * r2 : (m[o + i] + m[o + i + h]) * r2;
+  } else if (a.rot == 3) {
+    double acc = 0.0;
+    for (int e = 0; e < a.D; ++e) acc += (__popc(e & d) & 1) ? -m[e] : m[e];
+    mu = acc * (1.0 / sqrt(static_cast<double>(a.D)));
+  } else {
+    mu = m[d];
   }
-  a.k_mean[bh * a.D + d] = static_cast<float>(sum / static_cast<double>(a.N));
-  a.sv[bh * a.D + d] = __fdiv_rn(mx, 7.0f);
-  a.vinv[bh * a.D + d] = mx == 0.0f ? 0.0f : __fdiv_rn(7.0f, mx);
+  a.k_mean[bh * a.D + d] = static_cast<float>(mu);
 }
 
 // Pass 2: quantise.  Q, K: rotate (K also smoothed), per-token scale and codes.
@@ -617,7 +652,7 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_quant_kernel(PrologueArg
           a.sk[static_cast<size_t>(bh) * a.N + n] = __fdiv_rn(mk, 7.0f);
         }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) cacc[i] += static_cast<int>(bv[i] - 0x4B400000u);
+        for (int i = 0; i < 8; ++i) cacc[i] += static_cast<int>(bv[i] - (kQBits + 8u));
       }
     }
     __syncthreads();  // stage s consumed
@@ -700,6 +735,7 @@ WorkspaceLayout workspace_layout(const ra_problem& p) {
   const size_t bh = static_cast<size_t>(p.B) * p.H, T = rope_table_len(p), nc = prologue_nchunk(p);
   size_t o = 0;
   w.tab = o; o = align256(o + T * sizeof(float2));
+  w.tab0 = o; o = align256(o + T * sizeof(float2));
   w.ksum = o;  o = align256(o + bh * nc * p.D * sizeof(double));
   w.vmax = o;  o = align256(o + bh * nc * p.D * sizeof(float));
   w.vinv = o;  o = align256(o + bh * p.D * sizeof(float));
@@ -725,8 +761,8 @@ template <bool kBf16, int kRot, int kD>
 static cudaError_t launch_passes3(const PrologueArgs& a, dim3 grid, int red_bytes, int quant_bytes,
                                   cudaStream_t st) {
   cudaError_t e;
-  if ((e = set_smem(prologue_reduce_kernel<kBf16, kRot, kD>, red_bytes)) != cudaSuccess) return e;
-  prologue_reduce_kernel<kBf16, kRot, kD><<<grid, kThreads, red_bytes, st>>>(a);
+  if ((e = set_smem(prologue_reduce_kernel<kBf16, kD>, red_bytes)) != cudaSuccess) return e;
+  prologue_reduce_kernel<kBf16, kD><<<grid, kThreads, red_bytes, st>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   prologue_finalize_kernel<<<grid.y, 128, 0, st>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -755,6 +791,7 @@ cudaError_t launch_prologue(const ra_problem& p, int dtype, const void* q, const
   a.nchunk = prologue_nchunk(p);
   a.q = q; a.k = k; a.v = v; a.pos = pos;
   a.tab = reinterpret_cast<const float2*>(base + w.tab);
+  a.tab0 = reinterpret_cast<const float2*>(base + (p.rot == 1 ? w.tab0 : w.tab));
   a.ksum = reinterpret_cast<double*>(base + w.ksum);
   a.vmax = reinterpret_cast<float*>(base + w.vmax);
   a.vinv = reinterpret_cast<float*>(base + w.vinv);
@@ -762,6 +799,10 @@ cudaError_t launch_prologue(const ra_problem& p, int dtype, const void* q, const
   a.colsum = colsum;
   cudaError_t e = launch_tables(p, p.rot, reinterpret_cast<float2*>(base + w.tab), st);
   if (e != cudaSuccess) return e;
+  if (p.rot == 1) {  // the fused table differs from the plain one
+    e = launch_tables(p, 0, reinterpret_cast<float2*>(base + w.tab0), st);
+    if (e != cudaSuccess) return e;
+  }
   const dim3 grid(a.nchunk, p.B * p.H);
   // Dynamic shared memory: the staged sub-chunks (the reduce pass reuses it
   // for its per-thread partial sums, 12 bytes x 8 channels x threads).

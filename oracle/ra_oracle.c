@@ -26,9 +26,14 @@
  *   R2 RoPE is applied first, then the orthogonal rotation R (row vectors:
  *      x M R); H2 = [[1,1],[1,-1]]/sqrt(2).
  *   R3 K smoothing subtracts the per-channel mean over all N tokens of the
- *      rotated K; Q is not smoothed.
- *   R4 Q and K: per-token symmetric INT4, scale s = amax/7, code =
- *      clamp(rint(x * (7/amax)), -7, 7); amax = 0 gives s = 0 and codes 0.
+ *      rotated K; Q is not smoothed.  The mean is taken as R applied (in fp64)
+ *      to the fp64 mean of the RoPE'd K, which equals the mean of the rotated
+ *      K because R is linear and the same for every token; rounded once to
+ *      fp32.
+ *   R4 Q and K: per-token symmetric INT4, scale s = amax/7 (fp32), code =
+ *      clamp(rint(x * inv), -7, 7) with inv = fl(7/amax) and the product
+ *      x * inv taken exactly (one rounding, in the rint, ties to even);
+ *      amax = 0 gives s = 0 and codes 0.
  *   R5 V: per-channel symmetric INT4 over all N tokens, same rule.
  *   R6 P codes use the running row maximum after the current key block:
  *      c = clamp(rint(15 * exp(S - m)), 0, 15) - 8.
@@ -225,12 +230,48 @@ int orc_rope_rotate(const orc_problem* p, const float* x, const int32_t* pos,
   return ORC_OK;
 }
 
-/* Symmetric INT4 code of x given the reciprocal 7/amax (reading R4/R5). */
+/* The rotation R of rope_rotate_row applied to a D-vector in fp64 (no RoPE):
+ * interleaved: (m_2k +- m_2k+1)/sqrt2 on adjacent pairs; half: per segment
+ * (m_i +- m_i+h)/sqrt2 to positions 2i, 2i+1; full: m H_D / sqrt(D)
+ * (Sylvester, entry (-1)^popcount(e & d)); none: m. */
+static void rotate_mean(const orc_problem* p, const double* m, double* out) {
+  const int D = p->D;
+  const double r2 = 1.0 / sqrt(2.0);
+  if (p->rot == 1) {
+    for (int d = 0; d < D; d += 2) {
+      out[d] = (m[d] + m[d + 1]) * r2;
+      out[d + 1] = (m[d] - m[d + 1]) * r2;
+    }
+  } else if (p->rot == 2) {
+    int o = 0;
+    for (int j = 0; j < 3; ++j) {
+      const int h = p->seg[j] / 2;
+      for (int i = 0; i < h; ++i) {
+        out[o + 2 * i] = (m[o + i] + m[o + i + h]) * r2;
+        out[o + 2 * i + 1] = (m[o + i] - m[o + i + h]) * r2;
+      }
+      o += p->seg[j];
+    }
+  } else if (p->rot == 3) {
+    const double c = 1.0 / sqrt((double)D);
+    for (int d = 0; d < D; ++d) {
+      double acc = 0.0;
+      for (int e = 0; e < D; ++e) acc += (__builtin_popcount((unsigned)(e & d)) & 1) ? -m[e] : m[e];
+      out[d] = acc * c;
+    }
+  } else {
+    for (int d = 0; d < D; ++d) out[d] = m[d];
+  }
+}
+
+/* Symmetric INT4 code of x given the reciprocal inv = fl(7/amax) (reading
+ * R4/R5): rint, ties to even, of the exact product x * inv (two fp32 values:
+ * their product is exact in fp64). */
 static int quant4(float x, float inv) {
-  float y = x * inv;
-  float r = rintf(y);
-  if (r > 7.0f) r = 7.0f;
-  if (r < -7.0f) r = -7.0f;
+  double y = (double)x * (double)inv;
+  double r = rint(y);
+  if (r > 7.0) r = 7.0;
+  if (r < -7.0) r = -7.0;
   return (int)r;
 }
 
@@ -296,11 +337,28 @@ int orc_prologue_head(const orc_problem* p, const float* q, const float* k, cons
   for (int n = 0; n < N; ++n)
     rope_rotate_row(p, ta, tb, pos + 3 * n, k + (size_t)n * D, kr + (size_t)n * D, 0);
   if (k_rot) memcpy(k_rot, kr, sizeof(float) * (size_t)N * D);
-  /* K channel mean over all tokens: fp64 sum, rounded once to fp32 (reading R3). */
-  for (int d = 0; d < D; ++d) {
-    double s = 0.0;
-    for (int n = 0; n < N; ++n) s += (double)kr[(size_t)n * D + d];
-    kmean[d] = (float)(s / (double)N);
+  /* K channel mean over all tokens of the rotated K (reading R3): the rotation
+   * R is linear and the same for every token, so mean(x M_n R) = mean(x M_n) R.
+   * The mean of the RoPE'd K (no rotation) is summed in fp64, R is applied to
+   * that D-vector in fp64, and the result is rounded once to fp32. */
+  {
+    orc_problem p0 = *p;
+    p0.rot = 0;
+    float* ta0 = (float*)malloc(sizeof(float) * tl);
+    float* tb0 = (float*)malloc(sizeof(float) * tl);
+    orc_rope_tables(&p0, ta0, tb0);
+    double m[256], mr[256];
+    for (int d = 0; d < D; ++d) m[d] = 0.0;
+    for (int n = 0; n < N; ++n) {
+      float row[256];
+      rope_rotate_row(&p0, ta0, tb0, pos + 3 * n, k + (size_t)n * D, row, 0);
+      for (int d = 0; d < D; ++d) m[d] += (double)row[d];
+    }
+    for (int d = 0; d < D; ++d) m[d] /= (double)N;
+    rotate_mean(p, m, mr);
+    for (int d = 0; d < D; ++d) kmean[d] = (float)mr[d];
+    free(ta0);
+    free(tb0);
   }
   /* K: smooth, per-token quantise. */
 #pragma omp parallel for schedule(static)

@@ -35,6 +35,8 @@ and K -- RotateAttention, papernotes page, "key design 1"):
     128-point Sylvester Hadamard matrix: the offline V transform the pages
     absorb into W_v and W_o ("key design 3"), applied here to the synthetic V.
   * sharp=True multiplies Q by 8 (near one-hot softmax rows).
+  * rms_norm=False skips the normalisation (the recipe as literally stated,
+    used only to measure what the normalisation changes in the accuracy).
 
 bf16 tensors are produced from fp32 by round-to-nearest-even and returned as
 uint16 bit patterns so that both sides read exactly the same values.
@@ -66,6 +68,7 @@ class Workload:
     theta: float = 10000.0
     v_hadamard: bool = False
     sharp: bool = False
+    rms_norm: bool = True      # False: the literal recipe, without the per-row RMS normalisation
 
     @property
     def N(self) -> int:
@@ -179,8 +182,9 @@ def make_inputs(wl: Workload, heads: Tuple[int, ...] | None = None) -> Dict[str,
             q[:, ch] *= fac
             k[:, ch] *= fac
             k += rng.uniform(-3.0, 3.0, size=D).astype(np.float32)
-            q /= np.sqrt(np.mean(q * q, axis=1, keepdims=True, dtype=np.float32))
-            k /= np.sqrt(np.mean(k * k, axis=1, keepdims=True, dtype=np.float32))
+            if wl.rms_norm:
+                q /= np.sqrt(np.mean(q * q, axis=1, keepdims=True, dtype=np.float32))
+                k /= np.sqrt(np.mean(k * k, axis=1, keepdims=True, dtype=np.float32))
             if wl.dtype == "bf16":
                 vch = rng.choice(D, size=max(1, int(round(0.05 * D))), replace=False)
                 v[:, vch] *= 8.0

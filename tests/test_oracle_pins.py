@@ -233,6 +233,41 @@ def test_v_quantisation_round_trip(orc, name):
     assert np.array_equal(np.delete(h2["sv"], 3), np.delete(h["sv"], 3))
 
 
+def test_quantisation_rounds_the_exact_product_ties_to_even(orc):
+    """The INT4 decision is rint, ties to even, of the exact product
+    x * fl(7/amax) (a reading: the pages give code = round(x / s) without the
+    floating-point steps).  Expected codes come from exact rational arithmetic
+    here, not from the oracle: with amax = 7 the reciprocal is 1 and
+    2.5, 3.5, -0.5, 1.5, -2.5 are exact ties (to 2, 4, 0, 2, -2; rounding
+    half away from zero gives 3, 4, -1, 2, -3); with amax = 2.953125 the
+    exact product of 1.0546875 and fl(7/amax) is 2.50000002 (code 3), where
+    an fp32-rounded product would be the tie 2.5 (code 2)."""
+    from fractions import Fraction
+    sp = SPLITS[0]
+    p = orc.problem(D=sp["D"], seg=sp["seg"], grid=sp["grid"], rot=1, block_k=16)
+    pos = si.positions(sp["grid"])
+    N = len(pos)
+    v = np.zeros((N, sp["D"]), np.float32)
+    col0 = [2.953125, 1.0546875, -1.0546875]
+    col1 = [7.0, 2.5, 3.5, -0.5, 1.5, -2.5]
+    v[:len(col0), 0] = col0
+    v[:len(col1), 1] = col1
+    q = np.zeros((N, sp["D"]), np.float32)
+    h = orc.prologue_head(p, q, q, v, pos)
+    c = orc.unpack_codes(h["v4"]).astype(int)
+
+    def code(x, amax):
+        inv = np.float32(7.0) / np.float32(amax)          # fl(7/amax)
+        y = Fraction(float(np.float32(x))) * Fraction(float(inv))
+        r = round(y)                                        # Python rounds ties to even
+        return max(-7, min(7, r))
+
+    assert [code(x, col0[0]) for x in col0] == [7, 3, -3]
+    assert [code(x, 7.0) for x in col1] == [7, 2, 4, 0, 2, -2]
+    assert list(c[:len(col0), 0]) == [7, 3, -3]
+    assert list(c[:len(col1), 1]) == [7, 2, 4, 0, 2, -2]
+
+
 def test_k_mean_and_colsum(orc):
     wl, p, x, h = _head(orc, "small")
     mean = h["k_rot"].astype(np.float64).mean(axis=0)
@@ -401,6 +436,27 @@ def test_half_rotation_beats_no_rotation(orc):
         ref = orc.reference_attention_fp64(h["q_rot"], h["k_rot"], x["v"][0, 0])
         cos[rot] = _cosine(r["out"], ref)
     assert cos[2] > cos[0]
+
+
+def test_rotation_ranking_at_the_wan_shape(orc):
+    """At the Wan-like shape (N = 32760, segments 44/42/42), sampled query rows
+    of one head: half rotation beats no rotation and the full D x D Hadamard
+    beats both (papernotes page, main table and ablation on rotation
+    granularity), for the method's P codes and denominator."""
+    wl = si.WORKLOADS["wan"]
+    x = si.make_inputs(wl, heads=(0,))
+    q, k, v, pos = x["q"][0, 0], x["k"][0, 0], x["v"][0, 0], x["pos"]
+    p0 = orc.problem(wl.with_(rot=0))
+    rows = np.r_[0:128, wl.N - 128:wl.N]
+    ref = orc.reference_attention_fp64(orc.rope_rotate(p0, q, pos)[rows], orc.rope_rotate(p0, k, pos), v)
+    cos = {}
+    for rot in (0, 2, 3):
+        p = orc.problem(wl.with_(rot=rot))
+        h = orc.prologue_head(p, q, k, v, pos)
+        out = np.concatenate([orc.attention_int4_rows(p, h, 0, 128)["out"],
+                              orc.attention_int4_rows(p, h, wl.N - 128, wl.N)["out"]])
+        cos[rot] = _cosine(out, ref)
+    assert cos[2] > cos[0] and cos[3] > cos[2], cos
 
 
 def test_given_codes_entry(orc):
