@@ -30,7 +30,10 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "INT4 attn TOPS (4N²DH/t) & % INT8 tensor peak at N=32760,H=40,D=128"
-KERNELS_PER_STEP = 5  # rope table, channel reduce, finalize, quantise, attention
+# rope table (two for the interleaved rotation: the fused table and the plain
+# one the channel reduce uses), channel reduce, finalize, quantise, attention
+def kernels_per_step(rot: int) -> int:
+    return 6 if rot == 1 else 5
 # (name, p_mode, l_mode) of the attention's ablation switches timed after the step.
 ABLATIONS = (("fp32_l", 0, 1), ("local_max", 1, 0), ("local_max_fp32_l", 1, 1),
              ("symmetric_p", 2, 0), ("symmetric_p_fp32_l", 2, 1))
@@ -323,6 +326,40 @@ def run_ours(args, rank, world, local_rank):
     fb_ms = statistics.median(fb)
     del qr, kr, out_b
 
+    # The fused-Q step: the K/V-only prologue, then the attention kernel that
+    # quantises Q itself (no Q codes in HBM).  Timed like the step on the same
+    # inputs, after it; its output must equal the step's bit for bit.
+    fq = None
+    if wl.block_k == 64:
+        kv = ra.rope_rotate_quant(p, None, k, v, pos, workspace=ws)
+        out_f = torch.empty_like(out)
+        for _ in range(2):
+            ra.rope_rotate_quant(p, None, k, v, pos, out=kv, workspace=ws)
+            ra.attn_int4_qfused(p, q, pos, kv, out=out_f, workspace=ws)
+        torch.cuda.synchronize(dev)
+        fpro, fatt, fall = [], [], []
+        for _ in range(max(3, args.steps // 2)):
+            a0, a1, a2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            a0.record(stream)
+            ra.rope_rotate_quant(p, None, k, v, pos, out=kv, workspace=ws)
+            a1.record(stream)
+            ra.attn_int4_qfused(p, q, pos, kv, out=out_f, workspace=ws)
+            a2.record(stream)
+            torch.cuda.synchronize(dev)
+            fpro.append(a0.elapsed_time(a1))
+            fatt.append(a1.elapsed_time(a2))
+            fall.append(a0.elapsed_time(a2))
+        if ra.sync_status() != 0:
+            raise RuntimeError("device status not ok after the fused-Q step")
+        ra.rope_rotate_quant(p, q, k, v, pos, out=codes, workspace=ws)
+        ra.attn_int4(p, codes, out=out)
+        torch.cuda.synchronize(dev)
+        fq = {"ms_per_step": round(statistics.median(fall), 4),
+              "prologue_kv_ms": round(statistics.median(fpro), 4),
+              "attention_ms": round(statistics.median(fatt), 4),
+              "identical_to_step_output": bool(torch.equal(out_f.view(torch.int16), out.view(torch.int16)))}
+        del kv, out_f
+
     # The ablation switches of the attention (block-local max, symmetric P,
     # fp32 denominator), each timed on its own on the same codes; not part of
     # the INT4 step.
@@ -400,7 +437,8 @@ def run_ours(args, rank, world, local_rank):
         "ablations": {n: {"ms": round(t, 4), "tops": round(ops / (t * 1e-3) / 1e12, 1),
                           "frac": round(ops / (t * 1e-3) / 1e12 / int8_peak, 4)} for n, t in abl.items()},
         "prologue_by_rotation_ms": {n: round(t, 4) for n, t in rot_ms.items()},
-        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "fused_q": fq,
+        "gpu_launches": kernels_per_step(wl.rot) * args.steps,
         "clocks": clk.summary(),
     }
     return res

@@ -113,8 +113,10 @@ size_t ra_workspace_bytes(const ra_problem* p);
  *                  8 * v_colsum.
  *   workspace      device scratch of at least ra_workspace_bytes(p) bytes,
  *                  16-byte aligned; its contents on entry do not matter.
- * Quantisation: s = amax/7, code = clamp(rint(x * (7/amax)), -7, 7) in fp32;
- * amax = 0 gives s = 0 and codes 0.
+ * q, q4 and sq may all be NULL together: K and V only, for ra_attn_int4_qfused,
+ * which quantises Q itself (any other mix of NULLs is RA_ERR_INVALID_ARG).
+ * Quantisation: s = fl(amax/7), code = clamp(rint(x * fl(7/amax)), -7, 7) with
+ * the product taken exactly and ties to even; amax = 0 gives s = 0 and codes 0.
  */
 ra_status ra_rope_rotate_quant(const ra_problem* p, int in_dtype,
                                const void* q, const void* k, const void* v,
@@ -140,6 +142,30 @@ ra_status ra_attn_int4(const ra_problem* p,
                        const uint8_t* k4, const float* sk,
                        const uint8_t* v4, const float* sv,
                        void* out, float* lse, void* stream);
+
+/*
+ * INT4 attention with Q's prologue fused into the attention kernel (the
+ * papernotes page, highlights: the rotation rides on the elementwise RoPE
+ * pass at no extra memory traffic).  Instead of q4/sq, the kernel's code-
+ * widening warps read the raw Q, apply the same RoPE, rotation and per-token
+ * INT4 quantisation as ra_rope_rotate_quant (bit-identical codes and scales)
+ * and write the codes straight into the MMA's operand tiles; Q's codes never
+ * reach HBM.  K and V come from ra_rope_rotate_quant called with q, q4 and sq
+ * NULL.  Results equal ra_attn_int4 on the codes of the full prologue, bit for
+ * bit.
+ *   in_dtype   RA_DT_BF16 or RA_DT_F32: element type of q.
+ *   q          [B, H, N, D] raw Q (before RoPE).
+ *   pos        [N, 3] int32 grid positions (the same array as the prologue's).
+ *   k4, sk, v4, sv   as for ra_attn_int4 (from the K/V-only prologue).
+ *   workspace  device scratch of at least ra_workspace_bytes(p) bytes (the
+ *              RoPE table of p->rot is built in it; it may be the prologue's).
+ *   out, lse   as for ra_attn_int4.
+ * Implemented for block_k = 64 (D = 64 or 128) and the method's P codes and
+ * denominator; other block sizes return RA_ERR_UNSUPPORTED.
+ */
+ra_status ra_attn_int4_qfused(const ra_problem* p, int in_dtype, const void* q, const int32_t* pos,
+                              const uint8_t* k4, const float* sk, const uint8_t* v4, const float* sv,
+                              void* workspace, size_t ws_bytes, void* out, float* lse, void* stream);
 
 /*
  * Test entry on raw codes: runs the INT4 attention kernel of ra_attn_int4 on

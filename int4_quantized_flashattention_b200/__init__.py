@@ -17,7 +17,7 @@ import torch
 __all__ = [
     "ROT_NONE", "ROT_INTERLEAVED", "ROT_HALF", "ROT_FULL", "RaError", "Problem", "lib", "workspace_bytes",
     "rope_rotate_quant", "attn_int4", "test_int4_codes", "rope_bf16", "attn_bf16_fallback",
-    "sync_status", "library_path", "AttnOpts", "P_RANGE", "P_LOCAL_MAX", "P_SYMMETRIC", "L_CODES", "L_FP32",
+    "attn_int4_qfused", "sync_status", "library_path", "AttnOpts", "P_RANGE", "P_LOCAL_MAX", "P_SYMMETRIC", "L_CODES", "L_FP32",
 ]
 
 ROT_NONE, ROT_INTERLEAVED, ROT_HALF, ROT_FULL = 0, 1, 2, 3
@@ -82,9 +82,11 @@ def lib():
         L.ra_test_int4_codes_opts.argtypes = [P, vp] + [vp] * 6 + [C.c_int] * 3 + [vp] * 6
         L.ra_rope_bf16.argtypes = [P, C.c_int] + [vp] * 6 + [sz, vp]
         L.ra_attn_bf16_fallback.argtypes = [P] + [vp] * 6
+        L.ra_attn_int4_qfused.argtypes = [P, C.c_int] + [vp] * 7 + [sz] + [vp] * 3
         L.ra_sync_status.argtypes = [vp]
         for name in ("ra_rope_rotate_quant", "ra_attn_int4", "ra_test_int4_codes", "ra_rope_bf16",
-                     "ra_attn_bf16_fallback", "ra_sync_status", "ra_attn_int4_opts", "ra_test_int4_codes_opts"):
+                     "ra_attn_bf16_fallback", "ra_sync_status", "ra_attn_int4_opts", "ra_test_int4_codes_opts",
+                     "ra_attn_int4_qfused"):
             getattr(L, name).restype = C.c_int
         _lib = L
     return _lib
@@ -133,31 +135,34 @@ def _nblocks(p: Problem) -> int:
     return (p.N + p.block_k - 1) // p.block_k
 
 
-def rope_rotate_quant(p: Problem, q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, pos: torch.Tensor,
+def rope_rotate_quant(p: Problem, q: Optional[torch.Tensor], k: torch.Tensor, v: torch.Tensor, pos: torch.Tensor,
                       out: Optional[Dict[str, torch.Tensor]] = None, workspace: Optional[torch.Tensor] = None,
                       stream=None) -> Dict[str, torch.Tensor]:
-    """ra_rope_rotate_quant: returns q4, sq, k4, sk, k_mean, v4, sv, v_colsum."""
+    """ra_rope_rotate_quant: returns q4, sq, k4, sk, k_mean, v4, sv, v_colsum.
+    q = None runs K and V only (for attn_int4_qfused); q4 and sq are then absent."""
     B, H, N, D = p.B, p.H, p.N, p.D
-    dev = q.device
+    dev = k.device
     if out is None:
-        out = {
+        out = {} if q is None else {
             "q4": torch.empty(B, H, N, D // 2, dtype=torch.uint8, device=dev),
-            "sq": torch.empty(B, H, N, dtype=torch.float32, device=dev),
+            "sq": torch.empty(B, H, N, dtype=torch.float32, device=dev)}
+        out.update({
             "k4": torch.empty(B, H, N, D // 2, dtype=torch.uint8, device=dev),
             "sk": torch.empty(B, H, N, dtype=torch.float32, device=dev),
             "k_mean": torch.empty(B, H, D, dtype=torch.float32, device=dev),
             "v4": torch.empty(B, H, N, D // 2, dtype=torch.uint8, device=dev),
             "sv": torch.empty(B, H, D, dtype=torch.float32, device=dev),
             "v_colsum": torch.empty(B, H, _nblocks(p), D, dtype=torch.int32, device=dev),
-        }
+        })
     if workspace is None:
         workspace = torch.empty(max(workspace_bytes(p), 16), dtype=torch.uint8, device=dev)
-    dt = _in_dtype(q)
+    dt = _in_dtype(k)
     shp = (B, H, N, D)
     rc = lib().ra_rope_rotate_quant(
-        C.byref(p), dt, _ptr(q, q.dtype, shp, "q"), _ptr(k, q.dtype, shp, "k"), _ptr(v, q.dtype, shp, "v"),
+        C.byref(p), dt, _ptr(q, k.dtype, shp, "q"), _ptr(k, k.dtype, shp, "k"), _ptr(v, k.dtype, shp, "v"),
         _ptr(pos, torch.int32, (N, 3), "pos"),
-        _ptr(out["q4"], torch.uint8, (B, H, N, D // 2)), _ptr(out["sq"], torch.float32, (B, H, N)),
+        _ptr(out.get("q4") if q is not None else None, torch.uint8, (B, H, N, D // 2)),
+        _ptr(out.get("sq") if q is not None else None, torch.float32, (B, H, N)),
         _ptr(out["k4"], torch.uint8, (B, H, N, D // 2)), _ptr(out["sk"], torch.float32, (B, H, N)),
         _ptr(out["k_mean"], torch.float32, (B, H, D)), _ptr(out["v4"], torch.uint8, (B, H, N, D // 2)),
         _ptr(out["sv"], torch.float32, (B, H, D)), _ptr(out["v_colsum"], torch.int32, (B, H, _nblocks(p), D)),
@@ -181,6 +186,28 @@ def attn_int4(p: Problem, codes: Dict[str, torch.Tensor], out: Optional[torch.Te
         _ptr(out, torch.bfloat16, (B, H, N, D), "out"), _ptr(lse, torch.float32, (B, H, N), "lse"),
         C.c_void_p(_stream(stream)))
     _check("ra_attn_int4_opts", rc)
+    return out
+
+
+def attn_int4_qfused(p: Problem, q: torch.Tensor, pos: torch.Tensor, codes: Dict[str, torch.Tensor],
+                     out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                     workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """ra_attn_int4_qfused: INT4 attention that quantises the raw Q itself;
+    codes holds k4, sk, v4, sv (rope_rotate_quant with q = None).  Returns out."""
+    B, H, N, D = p.B, p.H, p.N, p.D
+    dev = q.device
+    if out is None:
+        out = torch.empty(B, H, N, D, dtype=torch.bfloat16, device=dev)
+    if workspace is None:
+        workspace = torch.empty(max(workspace_bytes(p), 16), dtype=torch.uint8, device=dev)
+    rc = lib().ra_attn_int4_qfused(
+        C.byref(p), _in_dtype(q), _ptr(q, q.dtype, (B, H, N, D), "q"), _ptr(pos, torch.int32, (N, 3), "pos"),
+        _ptr(codes["k4"], torch.uint8, (B, H, N, D // 2)), _ptr(codes["sk"], torch.float32, (B, H, N)),
+        _ptr(codes["v4"], torch.uint8, (B, H, N, D // 2)), _ptr(codes["sv"], torch.float32, (B, H, D)),
+        _ptr(workspace, torch.uint8), C.c_size_t(workspace.numel()),
+        _ptr(out, torch.bfloat16, (B, H, N, D), "out"), _ptr(lse, torch.float32, (B, H, N), "lse"),
+        C.c_void_p(_stream(stream)))
+    _check("ra_attn_int4_qfused", rc)
     return out
 
 

@@ -40,6 +40,7 @@
 
 #include "ra_common.cuh"
 #include "ra_internal.h"
+#include "ra_rope.cuh"
 
 namespace ra {
 namespace {
@@ -76,7 +77,13 @@ struct Cfg {
   static constexpr int kFRow = D / 4 + 4;                 // floats per thread (padded)
   static constexpr int oF = oKsc + kKS * BN * 4;
   static constexpr int oBar = oF + kTiles * 2 * kRows * kFRow * 4;
-  static constexpr int kNumBars = 4 + 2 * kPS + 2 * kKS + 2 * kVS + 4 + 4 + 4 + 2;
+  static constexpr int kNumBars = 4 + 2 * kPS + 2 * kKS + 2 * kVS + 4 + 4 + 4 + 2 + 2;
+  // Fused-Q path: the packed-Q staging area is free; it holds the half
+  // rotation's row exchange (16 token rows of D floats) and then the per-row
+  // Q scales of the two tiles.
+  static constexpr int oQx = oQPk;
+  static constexpr int oSq = oQPk + 16 * D * 4;
+  static_assert(16 * D * 4 + kTiles * kRows * 4 <= kTiles * kQPkBytes, "fused-Q scratch");
   static constexpr int oMisc = oBar + kNumBars * 8;
   static constexpr int kSmem = oMisc + 16 + 1024;       // + alignment slack
   static constexpr int kKwStride = ((kKwBytes + 1023) / 1024) * 1024;
@@ -97,6 +104,8 @@ struct Bars {
   uint64_t* p_full;   // [tile][buf]
   uint64_t* pv_done;  // [tile][buf]: P.V of the blocks whose P sits in S buffer buf
   uint64_t* drain;    // [issuer]
+  uint64_t* sq_full;  // fused Q: the item's per-row Q scales are in shared memory
+  uint64_t* sq_empty; // fused Q: every softmax warp has read them
 };
 
 struct AttnParams {
@@ -112,6 +121,12 @@ struct AttnParams {
   int32_t* dump_s;
   int8_t* dump_p;
   int32_t* dump_acc;
+  // fused-Q variant: raw Q [BH, N, D] (bf16 or fp32), positions, RoPE table
+  const void* qraw;
+  int qdtype, rot;
+  const int32_t* pos;
+  const float2* tab;
+  SegInfo seg;
 };
 
 // Widens one 16-byte chunk of packed codes (32 channels) into two 16-byte
@@ -181,6 +196,67 @@ __device__ __forceinline__ float tree_max(const float* x) {
 
 __device__ __forceinline__ void set_status(uint32_t bits) { atomicOr(&g_attn_status, bits); }
 
+// Fused Q of one item (query tiles 2 pair and 2 pair + 1 of head bh), by the
+// 128 widening threads: the prologue's per-token arithmetic (RoPE, rotation,
+// amax, 7/amax, one f32x2 FMA per code pair, shared through ra_rope.cuh, so
+// the codes and scales are bit-identical to ra_rope_rotate_quant's), written
+// straight into the widened s8 layout of the Q tiles (16 x code; per 32
+// channels the even ones, then the odd ones; 128B/64B swizzle) and the per-row
+// scales amax/7 into sqs[tile * 128 + row].  D/8 threads per row; rows past N
+// get codes 0 and scale 0.  Every lane runs every pass (the shuffles and the
+// half rotation's warp synchronisation are unconditional).
+template <int D>
+__device__ __forceinline__ void fused_q_item(const AttnParams& prm, uint8_t* qw, float* rows, float* sqs, int bh,
+                                             int pair, int wt) {
+  constexpr int lpt = D / 8;        // threads per row
+  constexpr int rpp = 128 / lpt;    // rows per pass
+  const int lane = wt & 31, wl = wt >> 5;
+  const int tok = wt / lpt, c0 = (wt % lpt) * 8;
+  float* const row = rows + (wl * (32 / lpt) + lane / lpt) * D;   // this row's exchange slot
+  RopePlan rp;
+  rp.init(prm.seg, c0);
+  const size_t head = static_cast<size_t>(bh) * prm.N * D;
+  const int pc = c0 >> 5, q4 = (c0 & 31) >> 3;
+  constexpr uint32_t kRep4 = kQBits * 0x01010101u;   // sum_i 256^i 0x4B400000 mod 2^32
+  for (int base = 0; base < kTiles * kRows; base += rpp) {
+    const int rr = base + tok;
+    const int tt = rr / kRows, r = rr % kRows;
+    const int n = (pair * kTiles + tt) * kRows + r;
+    const bool valid = n < prm.N;
+    float x[8];
+    int gp[3] = {0, 0, 0};
+    if (valid) {
+      load8(prm.qraw, head + static_cast<size_t>(n) * D + c0, prm.qdtype, x);
+#pragma unroll
+      for (int j = 0; j < 3; ++j) gp[j] = __ldg(prm.pos + 3 * n + j);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) x[i] = 0.0f;
+    }
+    float2 cf[4];
+    rope_coef8p(prm.seg, rp, prm.tab, gp, cf, &g_attn_status);
+    rope_apply8(prm.seg, rp, prm.rot, cf, c0, x, row);
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(x[i]));
+    m = group_max(m, lpt);
+    const float inv = m == 0.0f ? 0.0f : __fdiv_rn(7.0f, m);
+    uint32_t b[8];
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) quant4_bits2(x[i], x[i + 1], inv, inv, b + i);
+    // bytes code + 8 of the even / odd channels, then 16 x code as s8
+    uint32_t we = b[6], wo = b[7];
+    we = we * 256u + b[4]; we = we * 256u + b[2]; we = we * 256u + b[0];
+    wo = wo * 256u + b[5]; wo = wo * 256u + b[3]; wo = wo * 256u + b[1];
+    we = ((we - kRep4) << 4) ^ 0x80808080u;
+    wo = ((wo - kRep4) << 4) ^ 0x80808080u;
+    uint8_t* tile = qw + tt * (kRows * D);
+    *reinterpret_cast<uint32_t*>(tile + swz_offset(r, 2 * pc, D) + 4 * q4) = we;
+    *reinterpret_cast<uint32_t*>(tile + swz_offset(r, 2 * pc + 1, D) + 4 * q4) = wo;
+    if (c0 == 0) sqs[rr] = valid ? __fdiv_rn(m, 7.0f) : 0.0f;
+  }
+}
+
 // Records the first wait that gave up (site id, block counter, CTA) for diagnosis.
 __device__ __forceinline__ void note_timeout(uint32_t site, uint32_t g) {
   atomicCAS(&g_attn_diag, 0u, (site << 24) | ((g & 0xFFFFu) << 8) | (blockIdx.x & 0xFFu));
@@ -194,12 +270,14 @@ __device__ __forceinline__ bool wait_at(uint64_t* bar, uint32_t parity, volatile
 }
 
 // MODE bits 0-1: P codes (0 range-rectified, 1 block-local maximum, 2
-// symmetric); bit 2: fp32 denominator.
+// symmetric); bit 2: fp32 denominator; bit 3: fused Q (the widening warps
+// compute Q's codes and scales from the raw Q instead of loading them).
 template <int D, int BN, bool DUMP, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const AttnParams prm) {
   using C = Cfg<D, BN>;
+  constexpr bool kFQ = (MODE & 8) != 0;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base; pointer arithmetic on the shared array keeps the
   // shared address space visible to the compiler (LDS/STS, not generic LD/ST).
@@ -213,6 +291,7 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     B.kw_full = b; b += C::kKS; B.kw_empty = b; b += C::kKS;
     B.vw_full = b; b += C::kVS; B.vw_empty = b; b += C::kVS;
     B.s_full = b; b += 4; B.p_full = b; b += 4; B.pv_done = b; b += 4; B.drain = b; b += 2;
+    B.sq_full = b++; B.sq_empty = b++;
   }
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::oMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::oMisc + 4);
@@ -226,6 +305,8 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     for (int s = 0; s < 4; ++s) { mbar_init(B.s_full + s, 1); mbar_init(B.p_full + s, 8); mbar_init(B.pv_done + s, 1); }
     mbar_init(B.drain, 1);
     mbar_init(B.drain + 1, 1);
+    mbar_init(B.sq_full, 4);
+    mbar_init(B.sq_empty, 16);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -256,11 +337,13 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         bool ok = true;
         for (int item = blockIdx.x; item < prm.nitems && ok; item += gridDim.x, ++li) {
           const int bh = item / prm.npairs, pair = item % prm.npairs;
-          ok = wait_at(B.qpk_empty, (li & 1) ^ 1, abort_flag, 1u, li, 256u);
-          if (!ok) break;
-          mbar_arrive_expect_tx(B.qpk_full, kTiles * C::kQPkBytes);
-          for (int tt = 0; tt < kTiles; ++tt)
-            tma_load_3d(smem + C::oQPk + tt * C::kQPkBytes, &tm_q, B.qpk_full, 0, pair * 2 * kRows + tt * kRows, bh);
+          if constexpr (!kFQ) {
+            ok = wait_at(B.qpk_empty, (li & 1) ^ 1, abort_flag, 1u, li, 256u);
+            if (!ok) break;
+            mbar_arrive_expect_tx(B.qpk_full, kTiles * C::kQPkBytes);
+            for (int tt = 0; tt < kTiles; ++tt)
+              tma_load_3d(smem + C::oQPk + tt * C::kQPkBytes, &tm_q, B.qpk_full, 0, pair * 2 * kRows + tt * kRows, bh);
+          }
           for (int t = 0; t < nb; ++t, ++g) {
             const int s = g % C::kPS;
             ok = wait_at(B.pk_empty + s, ((g / C::kPS) & 1) ^ 1, abort_flag, 14u, g, 256u);
@@ -355,13 +438,25 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       bool ok = true;
       for (int item = blockIdx.x; item < prm.nitems && ok; item += gridDim.x, ++li) {
         const int bh = item / prm.npairs;
-        if (!(ok = wait_at(B.qpk_full, li & 1, abort_flag, 7u, li, 256u))) break;
-        if (!(ok = wait_at(B.q_free, (li & 1) ^ 1, abort_flag, 8u, li, 256u))) break;
-        for (int tt = 0; tt < kTiles; ++tt)
-          widen_tile<D>(smem + C::oQPk + tt * C::kQPkBytes, smem + C::oQ + tt * C::kQBytes, kRows, wt, 128);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) { mbar_arrive(B.qpk_empty); mbar_arrive(B.q_full); }
+        if constexpr (kFQ) {
+          // Q of the item from the raw input: the previous item's QK products
+          // are issued (q_free) and its Q scales read by every softmax warp.
+          if (!(ok = wait_at(B.q_free, (li & 1) ^ 1, abort_flag, 8u, li, 256u))) break;
+          if (!(ok = wait_at(B.sq_empty, (li & 1) ^ 1, abort_flag, 20u, li, 256u))) break;
+          fused_q_item<D>(prm, smem + C::oQ, reinterpret_cast<float*>(smem + C::oQx),
+                          reinterpret_cast<float*>(smem + C::oSq), bh, item % prm.npairs, wt);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) { mbar_arrive(B.q_full); mbar_arrive(B.sq_full); }
+        } else {
+          if (!(ok = wait_at(B.qpk_full, li & 1, abort_flag, 7u, li, 256u))) break;
+          if (!(ok = wait_at(B.q_free, (li & 1) ^ 1, abort_flag, 8u, li, 256u))) break;
+          for (int tt = 0; tt < kTiles; ++tt)
+            widen_tile<D>(smem + C::oQPk + tt * C::kQPkBytes, smem + C::oQ + tt * C::kQBytes, kRows, wt, 128);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) { mbar_arrive(B.qpk_empty); mbar_arrive(B.q_full); }
+        }
         for (int t = 0; t < nb; ++t, ++g) {
           const int s = g % C::kPS, ks = g % C::kKS, vs = g % C::kVS;
           if (!(ok = wait_at(B.pk_full + s, (g / C::kPS) & 1, abort_flag, 9u, g, 128u))) break;
@@ -475,12 +570,22 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
       for (int c = 0; c < kHD; c += 32) tmem_st_h<32, kHD>(tA + c, m);
     }
-    for (int item = blockIdx.x; item < prm.nitems && ok; item += gridDim.x) {
+    uint32_t li = 0;
+    for (int item = blockIdx.x; item < prm.nitems && ok; item += gridDim.x, ++li) {
       const int bh = item / prm.npairs, pair = item % prm.npairs;
       const int qtile = pair * 2 + tt;
       const int row = qtile * kRows + r;
       const bool row_ok = row < prm.N;
-      const float ci = row_ok ? __fmul_rn(prm.sq[static_cast<size_t>(bh) * prm.N + row], prm.inv_sqrt_d) : 0.0f;
+      float sq_row = 0.0f;
+      if constexpr (kFQ) {
+        if (!(ok = wait_at(B.sq_full, li & 1, abort_flag, 21u, li))) break;
+        sq_row = reinterpret_cast<const float*>(smem + C::oSq)[tt * kRows + r];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(B.sq_empty);
+      } else if (row_ok) {
+        sq_row = prm.sq[static_cast<size_t>(bh) * prm.N + row];
+      }
+      const float ci = row_ok ? __fmul_rn(sq_row, prm.inv_sqrt_d) : 0.0f;
       const float cpi = __fmul_rn(ci, kLog2e);
       const float2 cpi2 = make_float2(cpi, cpi);
       const bool dump_tile = DUMP && bh == prm.dump_bh && qtile == prm.dump_tile && row_ok;
@@ -752,7 +857,8 @@ cudaError_t launch_cfg(const ra_problem& p, const uint8_t* q4, const uint8_t* k4
 
 cudaError_t launch_attn_int4(const ra_problem& p, const uint8_t* q4, const float* sq, const uint8_t* k4,
                              const float* sk, const uint8_t* v4, const float* sv, void* out, float* lse,
-                             const AttnDump* dump, int mode, cudaStream_t st, int* unsupported) {
+                             const AttnDump* dump, int mode, cudaStream_t st, int* unsupported,
+                             const FusedQ* fq) {
   AttnParams prm{};
   prm.N = p.N;
   prm.BH = p.B * p.H;
@@ -769,6 +875,18 @@ cudaError_t launch_attn_int4(const ra_problem& p, const uint8_t* q4, const float
     prm.dump_s = dump->s; prm.dump_p = dump->p; prm.dump_acc = dump->acc;
   }
   *unsupported = 0;
+  if (fq) {
+    // Fused Q: block_k = 64, the method's P codes and denominator, no dump.
+    // The unused Q tensor map is encoded over the K codes (never loaded).
+    if (p.block_k != 64 || mode != 0 || dmp) {
+      *unsupported = 1;
+      return cudaSuccess;
+    }
+    prm.qraw = fq->q; prm.qdtype = fq->dtype; prm.pos = fq->pos; prm.tab = fq->tab;
+    prm.rot = p.rot; prm.seg = seg_info(p);
+    return p.D == 128 ? launch_cfg<128, 64, false, 8>(p, k4, k4, v4, prm, st)
+                      : launch_cfg<64, 64, false, 8>(p, k4, k4, v4, prm, st);
+  }
   if (p.block_k == 128)
     return launch_attn_int4_pair(p, q4, sq, k4, sk, v4, sv, out, lse, dump, mode, st, unsupported);
 #define RA_CASE(DD, BB, MM)                                                                          \

@@ -63,12 +63,38 @@ ra_status ra_rope_rotate_quant(const ra_problem* p, int in_dtype, const void* q,
                                float* sk, float* k_mean, uint8_t* v4, float* sv, int32_t* v_colsum,
                                void* workspace, size_t ws_bytes, void* stream) {
   if (!valid_problem(p) || (in_dtype != RA_DT_F32 && in_dtype != RA_DT_BF16)) return RA_ERR_INVALID_ARG;
-  const void* ptrs[] = {q, k, v, pos, q4, sq, k4, sk, k_mean, v4, sv, v_colsum, workspace};
+  // Q, q4 and sq are either all given or all NULL (K and V only).
+  const bool no_q = !q && !q4 && !sq;
+  const void* ptrs[] = {k, v, pos, k4, sk, k_mean, v4, sv, v_colsum, workspace};
   for (const void* x : ptrs)
     if (!aligned16(x)) return RA_ERR_INVALID_ARG;
+  if (!no_q && (!aligned16(q) || !aligned16(q4) || !aligned16(sq))) return RA_ERR_INVALID_ARG;
   if (ws_bytes < ra::workspace_layout(*p).total) return RA_ERR_INVALID_ARG;
   return from_cuda(ra::launch_prologue(*p, in_dtype, q, k, v, pos, q4, sq, k4, sk, k_mean, v4, sv, v_colsum,
                                        workspace, static_cast<cudaStream_t>(stream)));
+}
+
+ra_status ra_attn_int4_qfused(const ra_problem* p, int in_dtype, const void* q, const int32_t* pos,
+                              const uint8_t* k4, const float* sk, const uint8_t* v4, const float* sv,
+                              void* workspace, size_t ws_bytes, void* out, float* lse, void* stream) {
+  if (!valid_problem(p) || (in_dtype != RA_DT_F32 && in_dtype != RA_DT_BF16)) return RA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, pos, k4, sk, v4, sv, workspace, out};
+  for (const void* x : ptrs)
+    if (!aligned16(x)) return RA_ERR_INVALID_ARG;
+  if (!aligned16_or_null(lse)) return RA_ERR_INVALID_ARG;
+  if (ws_bytes < ra::workspace_layout(*p).total) return RA_ERR_INVALID_ARG;
+  if (p->block_k != 64) return RA_ERR_UNSUPPORTED;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ra::FusedQ fq;
+  fq.q = q;
+  fq.dtype = in_dtype;
+  fq.pos = pos;
+  cudaError_t e = ra::launch_rope_table(*p, workspace, &fq.tab, st);
+  if (e != cudaSuccess) return from_cuda(e);
+  int unsupported = 0;
+  e = ra::launch_attn_int4(*p, nullptr, nullptr, k4, sk, v4, sv, out, lse, nullptr, 0, st, &unsupported, &fq);
+  if (unsupported) return RA_ERR_UNSUPPORTED;
+  return from_cuda(e);
 }
 
 // Kernel mode bits from the ablation options (0 = the method's defaults).

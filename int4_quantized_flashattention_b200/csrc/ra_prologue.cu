@@ -21,6 +21,7 @@
 
 #include "ra_common.cuh"
 #include "ra_internal.h"
+#include "ra_rope.cuh"
 
 namespace ra {
 namespace {
@@ -29,36 +30,6 @@ __device__ uint32_t g_prologue_status = 0;
 
 constexpr int kThreads = 256;
 constexpr int kChunk = 256;  // tokens per CTA; a multiple of every block_k
-
-struct SegInfo {
-  int off[3];     // first channel of each segment
-  int dj[3];      // channels of each segment
-  int toff[3];    // first table entry of each segment
-  int grid[3];
-  int D;
-  float hscale;   // fp32 rounding of 1/sqrt(D), the full rotation's scale
-};
-
-__device__ __forceinline__ void load8(const void* base, size_t elem_off, int dtype, float* x) {
-  if (dtype == 1) {
-    const uint4 u = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(base) + elem_off);
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      x[2 * i] = __uint_as_float(w[i] << 16);
-      x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
-  } else {
-    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(base) + elem_off);
-    const float4 a = p[0], b = p[1];
-    x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-    x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
-  }
-}
-
-__device__ __forceinline__ int seg_of(const SegInfo& s, int d) {
-  return d < s.off[1] ? 0 : (d < s.off[2] ? 1 : 2);
-}
 
 // Reads the token's grid position; a position outside the grid is reported and
 // clamped so every table access stays in bounds.
@@ -114,191 +85,6 @@ __device__ __forceinline__ void rope_rotate8(const SegInfo& s, const float2* tab
   }
 }
 
-// Eight channels of one token as loaded from memory: one 16-byte word for bf16,
-// two for fp32.  Loads use the read-only path.
-template <bool kBf16>
-struct Raw8 {
-  uint4 u[kBf16 ? 1 : 2];
-};
-
-template <bool kBf16>
-__device__ __forceinline__ void load_raw8(const void* base, size_t elem_off, Raw8<kBf16>& r) {
-  if constexpr (kBf16) {
-    r.u[0] = __ldg(reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(base) + elem_off));
-  } else {
-    const uint4* p = reinterpret_cast<const uint4*>(static_cast<const float*>(base) + elem_off);
-    r.u[0] = __ldg(p);
-    r.u[1] = __ldg(p + 1);
-  }
-}
-
-template <bool kBf16>
-__device__ __forceinline__ void unpack8(const Raw8<kBf16>& r, float* x) {
-  if constexpr (kBf16) {
-    const uint32_t w[4] = {r.u[0].x, r.u[0].y, r.u[0].z, r.u[0].w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      x[2 * i] = __uint_as_float(w[i] << 16);
-      x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
-  } else {
-    x[0] = __uint_as_float(r.u[0].x); x[1] = __uint_as_float(r.u[0].y);
-    x[2] = __uint_as_float(r.u[0].z); x[3] = __uint_as_float(r.u[0].w);
-    x[4] = __uint_as_float(r.u[1].x); x[5] = __uint_as_float(r.u[1].y);
-    x[6] = __uint_as_float(r.u[1].z); x[7] = __uint_as_float(r.u[1].w);
-  }
-}
-
-// Per-thread constants of the RoPE table lookup: the segment and the pair of
-// each of the thread's 4 channel pairs, computed once.
-struct RopePlan {
-  int seg[4], off[4], stride[4];
-  // Half rotation: output channel c0 + i reads channels u and w = u + Dj/2 of
-  // the RoPE'd row and takes their sum (even) or difference (odd):
-  // hx[i] = u | w << 8 | odd << 16.
-  uint32_t hx[8];
-  __device__ __forceinline__ void init(const SegInfo& s, int c0) {
-#pragma unroll
-    for (int pr = 0; pr < 4; ++pr) {
-      const int d = c0 + 2 * pr;
-      const int j = seg_of(s, d);
-      seg[pr] = j;
-      off[pr] = s.toff[j] + ((d - s.off[j]) >> 1);
-      stride[pr] = s.dj[j] >> 1;
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int d = c0 + i;
-      const int j = seg_of(s, d);
-      const uint32_t u = static_cast<uint32_t>(s.off[j] + ((d - s.off[j]) >> 1));
-      hx[i] = u | ((u + (s.dj[j] >> 1)) << 8) | (static_cast<uint32_t>((d - s.off[j]) & 1) << 16);
-    }
-  }
-};
-
-// Table coefficients (a, b) of the thread's 4 channel pairs for a token at grid
-// position gp (one position per segment; out-of-grid positions are reported
-// and clamped so every table access stays in bounds).
-__device__ __forceinline__ void rope_coef8p(const SegInfo& s, const RopePlan& rp, const float2* tab,
-                                            const int* gp, float* ca, float* cb) {
-  int g[3];
-#pragma unroll
-  for (int j = 0; j < 3; ++j) {
-    g[j] = gp[j];
-    if (g[j] < 0 || g[j] >= s.grid[j]) {
-      atomicOr(&g_prologue_status, kStatusBadPosition);
-      g[j] = g[j] < 0 ? 0 : s.grid[j] - 1;
-    }
-  }
-#pragma unroll
-  for (int pr = 0; pr < 4; ++pr) {
-    const int gj = rp.seg[pr] == 0 ? g[0] : (rp.seg[pr] == 1 ? g[1] : g[2]);
-    const int idx = rp.off[pr] + gj * rp.stride[pr];
-    const float2 ab = __ldg(tab + idx);
-    ca[pr] = ab.x;
-    cb[pr] = ab.y;
-  }
-}
-
-// Full rotation: the token row times H_D / sqrt(D) (Sylvester Hadamard), as
-// butterflies (a, b) -> (a + b, a - b) on channels d apart, d = 1, 2, ..., D/2
-// in that order, then one fp32 scaling.  The thread holds channels
-// [c0, c0 + 8): distances 1, 2, 4 are in its registers, distances 8 ... D/2
-// pair it with the lanes 1 ... D/16 apart in its token's lane group.
-__device__ __forceinline__ void hadamard8(const SegInfo& s, int c0, float* x) {
-#pragma unroll
-  for (int d = 1; d < 8; d <<= 1)
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      if (!(i & d)) {
-        const float a = x[i], b = x[i + d];
-        x[i] = __fadd_rn(a, b);
-        x[i + d] = __fsub_rn(a, b);
-      }
-  const int g = c0 >> 3;  // this thread's place among the token's D/8 lanes
-  for (int m = 1; m < (s.D >> 3); m <<= 1) {
-    const bool upper = (g & m) != 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float o = __shfl_xor_sync(0xFFFFFFFFu, x[i], m);
-      x[i] = upper ? __fsub_rn(o, x[i]) : __fadd_rn(x[i], o);
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < 8; ++i) x[i] = __fmul_rn(x[i], s.hscale);
-}
-
-// The same arithmetic as rope_rotate8, from coefficients already loaded (rot
-// 3: the full Hadamard rotation after the RoPE pairs).
-__device__ __forceinline__ void rope_apply8(const SegInfo& s, const RopePlan& rp, int rot, const float* ca,
-                                            const float* cb, int c0, float* x, float* row) {
-#pragma unroll
-  for (int pr = 0; pr < 4; ++pr) {
-    const float a = ca[pr], b = cb[pr];
-    const float x0 = x[2 * pr], x1 = x[2 * pr + 1];
-    if (rot == 1) {
-      x[2 * pr] = __fadd_rn(__fmul_rn(x0, a), __fmul_rn(x1, b));
-      x[2 * pr + 1] = __fsub_rn(__fmul_rn(x0, b), __fmul_rn(x1, a));
-    } else {
-      x[2 * pr] = __fsub_rn(__fmul_rn(x0, a), __fmul_rn(x1, b));
-      x[2 * pr + 1] = __fadd_rn(__fmul_rn(x0, b), __fmul_rn(x1, a));
-    }
-  }
-  if (rot == 2) {
-    const float r2 = 0.70710678118654752440f;  // fp32 rounding of 1/sqrt(2)
-#pragma unroll
-    for (int i = 0; i < 8; ++i) row[c0 + i] = x[i];
-    __syncwarp();
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint32_t h = rp.hx[i];
-      const float u = row[h & 0xFFu], w = row[(h >> 8) & 0xFFu];
-      x[i] = (h >> 16) ? __fmul_rn(__fsub_rn(u, w), r2) : __fmul_rn(__fadd_rn(u, w), r2);
-    }
-    __syncwarp();
-  }
-  if (rot == 3) hadamard8(s, c0, x);
-}
-
-
-// For two elements: the bits of 1.5 * 2^23 + 8 + rint(x * inv), i.e.
-// 0x4B400000 + (code + 8) with code + 8 in [1, 15].  One f32x2 fused
-// multiply-add: the product x * inv is exact inside the FMA and the single
-// rounding to the integer grid of [2^23, 2^24) (ties to even; the offset is
-// even) is the rint of the exact product.
-//   * No clamp is needed: inv = fl(7/amax) with |x| <= amax (the token's or
-//     channel's own maximum), so |x * inv| <= 7 (1 + 2^-23) < 7.5 and rint
-//     already lies in [-7, 7]; amax = 0 gives inv = 0 and code 0.
-//   * The exact product is the decision on purpose: an f32x2 multiply and an
-//     f32x2 add in sequence are fused by the compiler even when written with
-//     explicit round-to-nearest (measured: the codes of exact fp32 ties
-//     x * inv = k + 1/2 followed the unrounded product), so a two-rounding
-//     decision would need scalar operations at twice the instruction count.
-constexpr uint32_t kQBits = 0x4B400000u;       // bits of 1.5 * 2^23
-constexpr float kQMagic8 = 12582920.0f;        // 1.5 * 2^23 + 8
-__device__ __forceinline__ void quant4_bits2(float x0, float x1, float inv0, float inv1, uint32_t* b) {
-  const float2 t = __ffma2_rn(make_float2(x0, x1), make_float2(inv0, inv1), make_float2(kQMagic8, kQMagic8));
-  b[0] = __float_as_uint(t.x);
-  b[1] = __float_as_uint(t.y);
-}
-
-// Packs the nibbles of eight quant4_bits2 results, element 2t in the low
-// nibble: sum_i 16^i b_i (integer multiply-adds) minus the known sum of the
-// 0x4B400000 parts leaves the nibbles code + 8 (at most 15: no carries);
-// XOR with 8 in every nibble turns code + 8 into the two's complement code.
-constexpr uint32_t kQBitsRep = kQBits * 0x11111111u;   // sum_i 16^i 0x4B400000 mod 2^32
-__device__ __forceinline__ uint32_t pack8_bits(const uint32_t* b) {
-  uint32_t acc = b[7];
-#pragma unroll
-  for (int i = 6; i >= 0; --i) acc = acc * 16u + b[i];
-  return (acc - kQBitsRep) ^ 0x88888888u;
-}
-
-// Max over the D/8 threads of a token (a contiguous lane group of size lpt).
-__device__ __forceinline__ float group_max(float v, int lpt) {
-  for (int o = lpt >> 1; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
-  return v;
-}
 
 struct PrologueArgs {
   SegInfo s;
@@ -327,11 +113,15 @@ __global__ void rope_table_kernel(SegInfo s, int total, double theta, int rot, f
   const double freq = pow(theta, -2.0 * static_cast<double>(k) / static_cast<double>(s.dj[j]));
   const double phi = static_cast<double>(g) * freq;
   const double c = cos(phi), sn = sin(phi);
+  float a, b;
   if (rot == 1) {
-    tab[e] = make_float2(static_cast<float>((c + sn) / sqrt(2.0)), static_cast<float>((c - sn) / sqrt(2.0)));
+    a = static_cast<float>((c + sn) / sqrt(2.0));
+    b = static_cast<float>((c - sn) / sqrt(2.0));
   } else {
-    tab[e] = make_float2(static_cast<float>(c), static_cast<float>(sn));
+    a = static_cast<float>(c);
+    b = static_cast<float>(sn);
   }
+  tab[e] = make_float2(a, b);
 }
 
 // Rows of kSub tokens of the input tensors are staged in shared memory by bulk
@@ -387,7 +177,7 @@ template <bool kBf16, int kD>
 __global__ void __launch_bounds__(kThreads, 3) prologue_reduce_kernel(PrologueArgs a) {
   using IO = StageIO<kBf16, 2, kStgR>;
   constexpr int kRot = 0;
-  __shared__ float rows[1][4][128];   // (unused by the plain RoPE)
+  __shared__ __align__(16) float rows[1][4][128];   // (unused by the plain RoPE)
   __shared__ uint64_t full[kStgR];
   __shared__ int abort_flag;
   extern __shared__ __align__(128) uint8_t stg[];
@@ -423,7 +213,8 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_reduce_kernel(PrologueAr
     for (int ti = warp * tpw + tok_in_warp; ti - tok_in_warp < kSub; ti += step) {
       const int n = n0 + sc * kSub + ti;
       const bool valid = n < a.N;
-      float x[8], y[8], ca[4], cb[4];
+      float x[8], y[8];
+      float2 cf[4];
       int gp[3] = {0, 0, 0};
       if (valid) {
         Raw8<kBf16> rk, rv;
@@ -437,8 +228,8 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_reduce_kernel(PrologueAr
 #pragma unroll
         for (int i = 0; i < 8; ++i) { x[i] = 0.0f; y[i] = 0.0f; }
       }
-      rope_coef8p(a.s, rp, a.tab0, gp, ca, cb);
-      rope_apply8(a.s, rp, kRot, ca, cb, c0, x, row);
+      rope_coef8p(a.s, rp, a.tab0, gp, cf, &g_prologue_status);
+      rope_apply8(a.s, rp, kRot, cf, c0, x, row);
       if (valid) {
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
@@ -536,12 +327,15 @@ __global__ void prologue_finalize_kernel(PrologueArgs a) {
 // V: per-channel codes, column sums per key block.  Q and K of a token share
 // the RoPE coefficients; column sums are kept per thread while a warp stays in
 // one key block, then combined across the warp's tokens and added to shared
-// memory.
-template <bool kBf16, int kRot, int kD>
+// memory.  kQ = false leaves Q out (the attention kernel's fused-Q path
+// quantises Q itself): only K and V are staged and written.
+template <bool kBf16, int kRot, int kD, bool kQ>
 __global__ void __launch_bounds__(kThreads, 3) prologue_quant_kernel(PrologueArgs a) {
-  using IO = StageIO<kBf16, 3, kStgQ>;
+  constexpr int kNT = kQ ? 3 : 2;          // staged tensors
+  constexpr int iK = kQ ? 1 : 0, iV = iK + 1;
+  using IO = StageIO<kBf16, kNT, kStgQ>;
   // Row buffer of the half rotation's exchange (one token row per warp slot).
-  __shared__ float rows[kRot == 2 ? kThreads / 32 : 1][4][128];
+  __shared__ __align__(16) float rows[kRot == 2 ? kThreads / 32 : 1][4][128];
   __shared__ int csum[kChunk / 16][128];
   __shared__ uint64_t full[kStgQ];
   __shared__ int abort_flag;
@@ -556,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_quant_kernel(PrologueArg
   const int n0 = chunk * kChunk;
   const size_t head = static_cast<size_t>(bh) * a.N * kD;
   const size_t head4 = static_cast<size_t>(bh) * a.N * (kD / 2);
-  const void* src[3] = {a.q, a.k, a.v};
+  const void* src[3] = {kQ ? a.q : a.k, kQ ? a.k : a.v, a.v};
   RopePlan rp;
   rp.init(a.s, c0);
   for (int i = threadIdx.x; i < nblk * kD; i += kThreads) csum[i / kD][i % kD] = 0;
@@ -605,14 +399,17 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_quant_kernel(PrologueArg
         flush();
         cblk = blk;
       }
-      float xq[8], xk[8], xv[8], ca[4], cb[4];
+      float xq[8] = {}, xk[8], xv[8];
+      float2 cf[4];
       int gp[3] = {0, 0, 0};
       if (valid) {
         Raw8<kBf16> rq, rk, rv;
-        IO::read(stg, kD, s, 0, ti, c0, rq);
-        IO::read(stg, kD, s, 1, ti, c0, rk);
-        IO::read(stg, kD, s, 2, ti, c0, rv);
-        unpack8<kBf16>(rq, xq);
+        if constexpr (kQ) {
+          IO::read(stg, kD, s, 0, ti, c0, rq);
+          unpack8<kBf16>(rq, xq);
+        }
+        IO::read(stg, kD, s, iK, ti, c0, rk);
+        IO::read(stg, kD, s, iV, ti, c0, rv);
         unpack8<kBf16>(rk, xk);
         unpack8<kBf16>(rv, xv);
 #pragma unroll
@@ -621,9 +418,9 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_quant_kernel(PrologueArg
 #pragma unroll
         for (int i = 0; i < 8; ++i) { xq[i] = 0.0f; xk[i] = 0.0f; xv[i] = 0.0f; }
       }
-      rope_coef8p(a.s, rp, a.tab, gp, ca, cb);
-      rope_apply8(a.s, rp, kRot, ca, cb, c0, xq, row);
-      rope_apply8(a.s, rp, kRot, ca, cb, c0, xk, row);
+      rope_coef8p(a.s, rp, a.tab, gp, cf, &g_prologue_status);
+      if constexpr (kQ) rope_apply8(a.s, rp, kRot, cf, c0, xq, row);
+      rope_apply8(a.s, rp, kRot, cf, c0, xk, row);
       float mq = 0.0f, mk = 0.0f;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -631,24 +428,24 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_quant_kernel(PrologueArg
         mq = fmaxf(mq, fabsf(xq[i]));
         mk = fmaxf(mk, fabsf(xk[i]));
       }
-      mq = group_max(mq, lpt);
+      if constexpr (kQ) mq = group_max(mq, lpt);
       mk = group_max(mk, lpt);
-      uint32_t bq[8], bk[8], bv[8];
       const float iq = mq == 0.0f ? 0.0f : __fdiv_rn(7.0f, mq);
       const float ik = mk == 0.0f ? 0.0f : __fdiv_rn(7.0f, mk);
+      uint32_t bq[8], bk[8], bv[8];
 #pragma unroll
       for (int i = 0; i < 8; i += 2) {
-        quant4_bits2(xq[i], xq[i + 1], iq, iq, bq + i);
+        if constexpr (kQ) quant4_bits2(xq[i], xq[i + 1], iq, iq, bq + i);
         quant4_bits2(xk[i], xk[i + 1], ik, ik, bk + i);
         quant4_bits2(xv[i], xv[i + 1], vinv[i], vinv[i + 1], bv + i);
       }
       if (valid) {
         const size_t o4 = head4 + static_cast<size_t>(n) * (kD / 2) + (c0 >> 1);
-        *reinterpret_cast<uint32_t*>(a.q4 + o4) = pack8_bits(bq);
+        if constexpr (kQ) *reinterpret_cast<uint32_t*>(a.q4 + o4) = pack8_bits(bq);
         *reinterpret_cast<uint32_t*>(a.k4 + o4) = pack8_bits(bk);
         *reinterpret_cast<uint32_t*>(a.v4 + o4) = pack8_bits(bv);
         if (c0 == 0) {
-          a.sq[static_cast<size_t>(bh) * a.N + n] = __fdiv_rn(mq, 7.0f);
+          if constexpr (kQ) a.sq[static_cast<size_t>(bh) * a.N + n] = __fdiv_rn(mq, 7.0f);
           a.sk[static_cast<size_t>(bh) * a.N + n] = __fdiv_rn(mk, 7.0f);
         }
 #pragma unroll
@@ -702,6 +499,8 @@ __global__ void __launch_bounds__(kThreads) rope_bf16_kernel(PrologueArgs a, __n
   }
 }
 
+}  // namespace
+
 SegInfo seg_info(const ra_problem& p) {
   SegInfo s;
   int o = 0, t = 0;
@@ -717,8 +516,6 @@ SegInfo seg_info(const ra_problem& p) {
   s.hscale = static_cast<float>(1.0 / sqrt(static_cast<double>(p.D)));
   return s;
 }
-
-}  // namespace
 
 size_t rope_table_len(const ra_problem& p) {
   size_t t = 0;
@@ -766,8 +563,14 @@ static cudaError_t launch_passes3(const PrologueArgs& a, dim3 grid, int red_byte
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   prologue_finalize_kernel<<<grid.y, 128, 0, st>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if ((e = set_smem(prologue_quant_kernel<kBf16, kRot, kD>, quant_bytes)) != cudaSuccess) return e;
-  prologue_quant_kernel<kBf16, kRot, kD><<<grid, kThreads, quant_bytes, st>>>(a);
+  if (a.q) {
+    if ((e = set_smem(prologue_quant_kernel<kBf16, kRot, kD, true>, quant_bytes)) != cudaSuccess) return e;
+    prologue_quant_kernel<kBf16, kRot, kD, true><<<grid, kThreads, quant_bytes, st>>>(a);
+  } else {
+    const int kv_bytes = quant_bytes / 3 * 2;
+    if ((e = set_smem(prologue_quant_kernel<kBf16, kRot, kD, false>, kv_bytes)) != cudaSuccess) return e;
+    prologue_quant_kernel<kBf16, kRot, kD, false><<<grid, kThreads, kv_bytes, st>>>(a);
+  }
   return cudaGetLastError();
 }
 
@@ -821,6 +624,13 @@ cudaError_t launch_prologue(const ra_problem& p, int dtype, const void* q, const
       return cudaErrorInvalidValue;
   }
   return e;
+}
+
+cudaError_t launch_rope_table(const ra_problem& p, void* ws, const float2** tab, cudaStream_t st) {
+  const WorkspaceLayout w = workspace_layout(p);
+  float2* t = reinterpret_cast<float2*>(static_cast<char*>(ws) + w.tab);
+  *tab = t;
+  return launch_tables(p, p.rot, t, st);
 }
 
 cudaError_t launch_rope_bf16(const ra_problem& p, int dtype, const void* q, const void* k,

@@ -12,7 +12,8 @@ Workloads (all B=1; positions enumerate a frames x height x width grid):
   wan      H=40, grid 21x30x52 (N=32760),  D=128, segments 44/42/42, interleaved, bf16
   hunyuan  H=24, grid 33x45x80 (N=118800), D=128, segments 16/56/56, half,        bf16
   sweep-N  H=40, D=128, 44/42/42, N in {4096, 8192, 16384, 32760, 65536},
-           interleaved (sweepN) and half rotation (sweepN_half)
+           interleaved (sweepN) and half rotation (sweepN_half); sweepN_sharp
+           is the interleaved sweep with the sharp-P variant
 
 Outlier recipe (the pages report that after 3D RoPE the Q/K outliers sit inside
 each frame/height/width segment, mostly in its first half, and are shared by Q
@@ -110,6 +111,8 @@ for _i, _n in enumerate(sorted(SWEEP_GRIDS)):
     WORKLOADS[f"sweep{_n}"] = _sweep(_n, _i, ROT_INTERLEAVED)
     # the sweep in the other rotation mode (same tensors, same seed)
     WORKLOADS[f"sweep{_n}_half"] = _sweep(_n, _i, ROT_HALF).with_(name=f"sweep{_n}_half")
+    # the sharp-P variant (Q x8: near one-hot softmax rows), interleaved rotation
+    WORKLOADS[f"sweep{_n}_sharp"] = _sweep(_n, _i, ROT_INTERLEAVED).with_(name=f"sweep{_n}_sharp", sharp=True)
 
 
 def positions(grid: Tuple[int, int, int]) -> np.ndarray:

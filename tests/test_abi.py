@@ -10,6 +10,14 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "ra.h")
 
 
+def _no_gpu():
+    """Checks that pass validation and reach a launch use fake pointers: they
+    run only where no GPU is visible (the launch then fails with RA_ERR_CUDA)."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("reaches a launch with fake pointers; host-only check")
+
+
 def _declared():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
@@ -29,7 +37,7 @@ def test_header_declares_the_entry_points():
     names = _declared()
     for n in ("ra_rope_rotate_quant", "ra_attn_int4", "ra_attn_bf16_fallback", "ra_test_int4_codes",
               "ra_rope_bf16", "ra_workspace_bytes", "ra_sync_status", "ra_status_string",
-              "ra_attn_int4_opts", "ra_test_int4_codes_opts"):
+              "ra_attn_int4_opts", "ra_test_int4_codes_opts", "ra_attn_int4_qfused"):
         assert n in names
 
 
@@ -109,6 +117,7 @@ def test_block_k_128_is_dispatched(ra):
     """block_k = 128 (the CTA-pair kernel) passes validation and is not
     refused as unsupported, in every mode; without a GPU the launch itself
     then fails with RA_ERR_CUDA."""
+    _no_gpu()
     p = _wan(ra, block_k=128)
     good = C.c_void_p(0x10000)
     L = ra.lib()
@@ -143,3 +152,52 @@ def test_test_entry_rejects_bad_tile(ra):
     for b, h, t in ((1, 0, 0), (0, 40, 0), (0, 0, ntiles), (-1, 0, 0)):
         rc = L.ra_test_int4_codes(C.byref(p), *([good] * 6), b, h, t, None, None, None, good, None, None)
         assert rc == 1
+
+
+def test_qfused_entry_validates_before_any_launch(ra):
+    """ra_attn_int4_qfused: invalid problems, bad pointers or a short workspace
+    are RA_ERR_INVALID_ARG, block sizes other than 64 RA_ERR_UNSUPPORTED, all
+    before any launch (no GPU needed)."""
+    L = ra.lib()
+    good, bad = C.c_void_p(0x10000), C.c_void_p(0x10004)
+    p = _wan(ra)
+    need = ra.workspace_bytes(p)
+
+    def call(pp, dt=1, ptrs=None, ws=need, lse=None):
+        ptrs = ptrs or [good] * 6
+        return L.ra_attn_int4_qfused(C.byref(pp), dt, *ptrs[:6], good, C.c_size_t(ws), good, lse, None)
+    assert call(p, dt=7) == 1
+    for i in range(6):
+        ptrs = [good] * 6
+        ptrs[i] = bad
+        assert call(p, ptrs=ptrs) == 1
+        ptrs[i] = None
+        assert call(p, ptrs=ptrs) == 1
+    assert call(p, ws=need - 16) == 1
+    assert call(p, lse=bad) == 1
+    q = _wan(ra)
+    q.D = 96
+    assert call(q) == 1
+    assert call(_wan(ra, block_k=32)) == 2
+    assert call(_wan(ra, block_k=128)) == 2
+
+
+def test_kv_only_prologue_needs_all_three_q_pointers_null(ra):
+    """ra_rope_rotate_quant accepts q, q4 and sq all NULL (K and V only); a
+    partial set is RA_ERR_INVALID_ARG.  The full-NULL call passes validation
+    (without a GPU it then fails at the launch with RA_ERR_CUDA)."""
+    _no_gpu()
+    L = ra.lib()
+    good = C.c_void_p(0x10000)
+    p = _wan(ra)
+    need = C.c_size_t(ra.workspace_bytes(p))
+    base = [good] * 13
+    for drop in ((0,), (4,), (5,), (0, 4), (0, 5), (4, 5)):
+        args = list(base)
+        for i in drop:
+            args[i] = None
+        assert L.ra_rope_rotate_quant(C.byref(p), 1, *args, need, None) == 1, drop
+    args = list(base)
+    for i in (0, 4, 5):
+        args[i] = None
+    assert L.ra_rope_rotate_quant(C.byref(p), 1, *args, need, None) not in (1, 2)
