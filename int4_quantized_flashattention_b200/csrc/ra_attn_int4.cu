@@ -77,15 +77,13 @@ struct Cfg {
   static constexpr int kFRow = D / 4 + 4;                 // floats per thread (padded)
   static constexpr int oF = oKsc + kKS * BN * 4;
   static constexpr int oBar = oF + kTiles * 2 * kRows * kFRow * 4;
-  static constexpr int kNumBars = 4 + 2 * kPS + 2 * kKS + 2 * kVS + 4 + 4 + 4 + 2 + 2;
-  // Fused-Q path: the packed-Q staging area is free; it holds the half
-  // rotation's row exchange (16 token rows of D floats) and then the per-row
-  // Q scales of the two tiles.
-  static constexpr int oQx = oQPk;
-  static constexpr int oSq = oQPk + 16 * D * 4;
-  static_assert(16 * D * 4 + kTiles * kRows * 4 <= kTiles * kQPkBytes, "fused-Q scratch");
+  static constexpr int kNumBars = 4 + 2 * kPS + 2 * kKS + 2 * kVS + 4 + 4 + 4 + 2 + 4;
   static constexpr int oMisc = oBar + kNumBars * 8;
-  static constexpr int kSmem = oMisc + 16 + 1024;       // + alignment slack
+  // Fused-Q path: the Q warp's half-rotation row exchange (32 / (D/8) token
+  // rows of D floats = 1 KB) and a ring of two items' per-row Q scales.
+  static constexpr int oQx = oMisc + 64;
+  static constexpr int oSq = oQx + 1024;
+  static constexpr int kSmem = oSq + 2 * kTiles * kRows * 4 + 1024;   // + alignment slack
   static constexpr int kKwStride = ((kKwBytes + 1023) / 1024) * 1024;
   static constexpr int kVwStride = ((kVwBytes + 1023) / 1024) * 1024;
   static constexpr uint32_t kSwz = D == 128 ? kSwizzle128B : kSwizzle64B;
@@ -104,8 +102,8 @@ struct Bars {
   uint64_t* p_full;   // [tile][buf]
   uint64_t* pv_done;  // [tile][buf]: P.V of the blocks whose P sits in S buffer buf
   uint64_t* drain;    // [issuer]
-  uint64_t* sq_full;  // fused Q: the item's per-row Q scales are in shared memory
-  uint64_t* sq_empty; // fused Q: every softmax warp has read them
+  uint64_t* sq_full;  // [slot] fused Q: an item's per-row Q scales are in shared memory
+  uint64_t* sq_empty; // [slot] fused Q: every softmax warp has read them
 };
 
 struct AttnParams {
@@ -196,28 +194,26 @@ __device__ __forceinline__ float tree_max(const float* x) {
 
 __device__ __forceinline__ void set_status(uint32_t bits) { atomicOr(&g_attn_status, bits); }
 
-// Fused Q of one item (query tiles 2 pair and 2 pair + 1 of head bh), by the
-// 128 widening threads: the prologue's per-token arithmetic (RoPE, rotation,
-// amax, 7/amax, one f32x2 FMA per code pair, shared through ra_rope.cuh, so
-// the codes and scales are bit-identical to ra_rope_rotate_quant's), written
-// straight into the widened s8 layout of the Q tiles (16 x code; per 32
-// channels the even ones, then the odd ones; 128B/64B swizzle) and the per-row
-// scales amax/7 into sqs[tile * 128 + row].  D/8 threads per row; rows past N
-// get codes 0 and scale 0.  Every lane runs every pass (the shuffles and the
-// half rotation's warp synchronisation are unconditional).
+// Fused Q of one item (query tiles 2 pair and 2 pair + 1 of head bh), by one
+// warp: the prologue's per-token arithmetic (RoPE, rotation, amax, 7/amax, one
+// f32x2 FMA per code pair and the nibble packing, shared through ra_rope.cuh,
+// so the codes and scales are bit-identical to ra_rope_rotate_quant's),
+// written as packed rows into the packed-Q staging tiles (the layout the TMA
+// would load) and the per-row scales amax/7 into sqs[tile * 128 + row].  D/8
+// lanes per row, two rows per lane in flight; rows past N get codes 0 and
+// scale 0.  Every lane runs every pass (the shuffles and the half rotation's
+// warp synchronisation are unconditional).
 template <int D>
-__device__ __forceinline__ void fused_q_item(const AttnParams& prm, uint8_t* qw, float* rows, float* sqs, int bh,
-                                             int pair, int wt) {
-  constexpr int lpt = D / 8;        // threads per row
-  constexpr int rpp = 128 / lpt;    // rows per pass
-  const int lane = wt & 31, wl = wt >> 5;
-  const int tok = wt / lpt, c0 = (wt % lpt) * 8;
-  float* const row = rows + (wl * (32 / lpt) + lane / lpt) * D;   // this row's exchange slot
+__device__ __forceinline__ void fused_q_pack(const AttnParams& prm, uint8_t* qpk, float* rows, float* sqs, int bh,
+                                             int pair, int lane) {
+  constexpr int lpt = D / 8;        // lanes per row
+  constexpr int rpp = 32 / lpt;     // rows per pass
+  const int tok = lane / lpt, c0 = (lane % lpt) * 8;
+  float* const row = rows + tok * D;   // this row's exchange slot
   RopePlan rp;
   rp.init(prm.seg, c0);
   const size_t head = static_cast<size_t>(bh) * prm.N * D;
-  const int pc = c0 >> 5, q4 = (c0 & 31) >> 3;
-  constexpr uint32_t kRep4 = kQBits * 0x01010101u;   // sum_i 256^i 0x4B400000 mod 2^32
+#pragma unroll 2
   for (int base = 0; base < kTiles * kRows; base += rpp) {
     const int rr = base + tok;
     const int tt = rr / kRows, r = rr % kRows;
@@ -244,15 +240,7 @@ __device__ __forceinline__ void fused_q_item(const AttnParams& prm, uint8_t* qw,
     uint32_t b[8];
 #pragma unroll
     for (int i = 0; i < 8; i += 2) quant4_bits2(x[i], x[i + 1], inv, inv, b + i);
-    // bytes code + 8 of the even / odd channels, then 16 x code as s8
-    uint32_t we = b[6], wo = b[7];
-    we = we * 256u + b[4]; we = we * 256u + b[2]; we = we * 256u + b[0];
-    wo = wo * 256u + b[5]; wo = wo * 256u + b[3]; wo = wo * 256u + b[1];
-    we = ((we - kRep4) << 4) ^ 0x80808080u;
-    wo = ((wo - kRep4) << 4) ^ 0x80808080u;
-    uint8_t* tile = qw + tt * (kRows * D);
-    *reinterpret_cast<uint32_t*>(tile + swz_offset(r, 2 * pc, D) + 4 * q4) = we;
-    *reinterpret_cast<uint32_t*>(tile + swz_offset(r, 2 * pc + 1, D) + 4 * q4) = wo;
+    *reinterpret_cast<uint32_t*>(qpk + tt * (kRows * D / 2) + r * (D / 2) + (c0 >> 1)) = pack8_bits(b);
     if (c0 == 0) sqs[rr] = valid ? __fdiv_rn(m, 7.0f) : 0.0f;
   }
 }
@@ -270,8 +258,8 @@ __device__ __forceinline__ bool wait_at(uint64_t* bar, uint32_t parity, volatile
 }
 
 // MODE bits 0-1: P codes (0 range-rectified, 1 block-local maximum, 2
-// symmetric); bit 2: fp32 denominator; bit 3: fused Q (the widening warps
-// compute Q's codes and scales from the raw Q instead of loading them).
+// symmetric); bit 2: fp32 denominator; bit 3: fused Q (warp 3 computes Q's
+// packed codes and scales from the raw Q in place of the TMA load of q4).
 template <int D, int BN, bool DUMP, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -291,7 +279,7 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     B.kw_full = b; b += C::kKS; B.kw_empty = b; b += C::kKS;
     B.vw_full = b; b += C::kVS; B.vw_empty = b; b += C::kVS;
     B.s_full = b; b += 4; B.p_full = b; b += 4; B.pv_done = b; b += 4; B.drain = b; b += 2;
-    B.sq_full = b++; B.sq_empty = b++;
+    B.sq_full = b; b += 2; B.sq_empty = b; b += 2;
   }
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::oMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::oMisc + 4);
@@ -305,8 +293,7 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     for (int s = 0; s < 4; ++s) { mbar_init(B.s_full + s, 1); mbar_init(B.p_full + s, 8); mbar_init(B.pv_done + s, 1); }
     mbar_init(B.drain, 1);
     mbar_init(B.drain + 1, 1);
-    mbar_init(B.sq_full, 4);
-    mbar_init(B.sq_empty, 16);
+    for (int s = 0; s < 2; ++s) { mbar_init(B.sq_full + s, 1); mbar_init(B.sq_empty + s, 16); }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -429,6 +416,26 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         while (!mbar_try_wait(B.drain + tt, 0) && ++it < kSpinLimit) {}
         if (!ok) set_status(kStatusTimeout);
       }
+    } else if (warp == 3) {
+      // ------------------------------------------------------------ fused-Q warp
+      // Produces each item's packed Q (in place of the TMA load) and its
+      // per-row scales, as soon as the widening warps have consumed the
+      // previous item's packed Q: a whole item of slack.
+      if constexpr (kFQ) {
+        uint32_t li = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; item < prm.nitems && ok; item += gridDim.x, ++li) {
+          const uint32_t slot = li & 1;
+          if (!(ok = wait_at(B.qpk_empty, (li & 1) ^ 1, abort_flag, 22u, li, 256u))) break;
+          if (!(ok = wait_at(B.sq_empty + slot, ((li >> 1) & 1) ^ 1, abort_flag, 20u, li, 256u))) break;
+          fused_q_pack<D>(prm, smem + C::oQPk, reinterpret_cast<float*>(smem + C::oQx),
+                          reinterpret_cast<float*>(smem + C::oSq) + slot * kTiles * kRows, item / prm.npairs,
+                          item % prm.npairs, lane);
+          __syncwarp();
+          if (lane == 0) { mbar_arrive(B.qpk_full); mbar_arrive(B.sq_full + slot); }
+        }
+        if (!ok) set_status(kStatusTimeout);
+      }
     } else if (warp >= 4) {
       // ------------------------------------------------------------ widening warps
       const int wt = threadIdx.x - 128;  // 0..127
@@ -438,25 +445,15 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       bool ok = true;
       for (int item = blockIdx.x; item < prm.nitems && ok; item += gridDim.x, ++li) {
         const int bh = item / prm.npairs;
-        if constexpr (kFQ) {
-          // Q of the item from the raw input: the previous item's QK products
-          // are issued (q_free) and its Q scales read by every softmax warp.
-          if (!(ok = wait_at(B.q_free, (li & 1) ^ 1, abort_flag, 8u, li, 256u))) break;
-          if (!(ok = wait_at(B.sq_empty, (li & 1) ^ 1, abort_flag, 20u, li, 256u))) break;
-          fused_q_item<D>(prm, smem + C::oQ, reinterpret_cast<float*>(smem + C::oQx),
-                          reinterpret_cast<float*>(smem + C::oSq), bh, item % prm.npairs, wt);
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) { mbar_arrive(B.q_full); mbar_arrive(B.sq_full); }
-        } else {
-          if (!(ok = wait_at(B.qpk_full, li & 1, abort_flag, 7u, li, 256u))) break;
-          if (!(ok = wait_at(B.q_free, (li & 1) ^ 1, abort_flag, 8u, li, 256u))) break;
-          for (int tt = 0; tt < kTiles; ++tt)
-            widen_tile<D>(smem + C::oQPk + tt * C::kQPkBytes, smem + C::oQ + tt * C::kQBytes, kRows, wt, 128);
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) { mbar_arrive(B.qpk_empty); mbar_arrive(B.q_full); }
-        }
+        // The packed Q of the item (TMA, or the fused-Q warp) is widened once
+        // the previous item's QK products have been issued (q_free).
+        if (!(ok = wait_at(B.qpk_full, li & 1, abort_flag, 7u, li, 256u))) break;
+        if (!(ok = wait_at(B.q_free, (li & 1) ^ 1, abort_flag, 8u, li, 256u))) break;
+        for (int tt = 0; tt < kTiles; ++tt)
+          widen_tile<D>(smem + C::oQPk + tt * C::kQPkBytes, smem + C::oQ + tt * C::kQBytes, kRows, wt, 128);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) { mbar_arrive(B.qpk_empty); mbar_arrive(B.q_full); }
         for (int t = 0; t < nb; ++t, ++g) {
           const int s = g % C::kPS, ks = g % C::kKS, vs = g % C::kVS;
           if (!(ok = wait_at(B.pk_full + s, (g / C::kPS) & 1, abort_flag, 9u, g, 128u))) break;
@@ -578,10 +575,11 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
       const bool row_ok = row < prm.N;
       float sq_row = 0.0f;
       if constexpr (kFQ) {
-        if (!(ok = wait_at(B.sq_full, li & 1, abort_flag, 21u, li))) break;
-        sq_row = reinterpret_cast<const float*>(smem + C::oSq)[tt * kRows + r];
+        const uint32_t slot = li & 1;
+        if (!(ok = wait_at(B.sq_full + slot, (li >> 1) & 1, abort_flag, 21u, li))) break;
+        sq_row = reinterpret_cast<const float*>(smem + C::oSq)[(slot * kTiles + tt) * kRows + r];
         __syncwarp();
-        if (lane == 0) mbar_arrive(B.sq_empty);
+        if (lane == 0) mbar_arrive(B.sq_empty + slot);
       } else if (row_ok) {
         sq_row = prm.sq[static_cast<size_t>(bh) * prm.N + row];
       }
