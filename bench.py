@@ -360,6 +360,44 @@ def run_ours(args, rank, world, local_rank):
               "identical_to_step_output": bool(torch.equal(out_f.view(torch.int16), out.view(torch.int16)))}
         del kv, out_f
 
+    # The s8 code layout: the prologue writes one code per byte and the
+    # attention loads Q, K and V tiles by TMA straight into its MMA operands
+    # (no widening).  Timed like the step, after it; its output must equal
+    # the step's bit for bit.
+    s8 = None
+    if wl.block_k == 64:
+        c8 = ra.rope_rotate_quant_s8(p, q, k, v, pos, workspace=ws)
+        out_8 = torch.empty_like(out)
+        for _ in range(2):
+            ra.rope_rotate_quant_s8(p, q, k, v, pos, out=c8, workspace=ws)
+            ra.attn_int4_s8(p, c8, out=out_8)
+        torch.cuda.synchronize(dev)
+        spro, satt, sall = [], [], []
+        for _ in range(max(3, args.steps // 2)):
+            a0, a1, a2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            a0.record(stream)
+            ra.rope_rotate_quant_s8(p, q, k, v, pos, out=c8, workspace=ws)
+            a1.record(stream)
+            ra.attn_int4_s8(p, c8, out=out_8)
+            a2.record(stream)
+            torch.cuda.synchronize(dev)
+            spro.append(a0.elapsed_time(a1))
+            satt.append(a1.elapsed_time(a2))
+            sall.append(a0.elapsed_time(a2))
+        if ra.sync_status() != 0:
+            raise RuntimeError("device status not ok after the s8-layout step")
+        ra.rope_rotate_quant(p, q, k, v, pos, out=codes, workspace=ws)
+        ra.attn_int4(p, codes, out=out)
+        torch.cuda.synchronize(dev)
+        s8_att = statistics.median(satt)
+        s8 = {"ms_per_step": round(statistics.median(sall), 4),
+              "prologue_ms": round(statistics.median(spro), 4),
+              "attention_ms": round(s8_att, 4),
+              "attention_tops": round(wl.attn_ops() / (s8_att * 1e-3) / 1e12, 1),
+              "attention_frac": round(wl.attn_ops() / (s8_att * 1e-3) / 1e12 / (2.0 * _peaks()["bf16_tflops"]), 4),
+              "identical_to_step_output": bool(torch.equal(out_8.view(torch.int16), out.view(torch.int16)))}
+        del c8, out_8
+
     # The ablation switches of the attention (block-local max, symmetric P,
     # fp32 denominator), each timed on its own on the same codes; not part of
     # the INT4 step.
@@ -438,6 +476,7 @@ def run_ours(args, rank, world, local_rank):
                           "frac": round(ops / (t * 1e-3) / 1e12 / int8_peak, 4)} for n, t in abl.items()},
         "prologue_by_rotation_ms": {n: round(t, 4) for n, t in rot_ms.items()},
         "fused_q": fq,
+        "s8_layout": s8,
         "gpu_launches": kernels_per_step(wl.rot) * args.steps,
         "clocks": clk.summary(),
     }

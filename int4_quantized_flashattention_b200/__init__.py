@@ -17,7 +17,7 @@ import torch
 __all__ = [
     "ROT_NONE", "ROT_INTERLEAVED", "ROT_HALF", "ROT_FULL", "RaError", "Problem", "lib", "workspace_bytes",
     "rope_rotate_quant", "attn_int4", "test_int4_codes", "rope_bf16", "attn_bf16_fallback",
-    "attn_int4_qfused", "sync_status", "library_path", "AttnOpts", "P_RANGE", "P_LOCAL_MAX", "P_SYMMETRIC", "L_CODES", "L_FP32",
+    "attn_int4_qfused", "rope_rotate_quant_s8", "attn_int4_s8", "sync_status", "library_path", "AttnOpts", "P_RANGE", "P_LOCAL_MAX", "P_SYMMETRIC", "L_CODES", "L_FP32",
 ]
 
 ROT_NONE, ROT_INTERLEAVED, ROT_HALF, ROT_FULL = 0, 1, 2, 3
@@ -83,10 +83,12 @@ def lib():
         L.ra_rope_bf16.argtypes = [P, C.c_int] + [vp] * 6 + [sz, vp]
         L.ra_attn_bf16_fallback.argtypes = [P] + [vp] * 6
         L.ra_attn_int4_qfused.argtypes = [P, C.c_int] + [vp] * 7 + [sz] + [vp] * 3
+        L.ra_rope_rotate_quant_s8.argtypes = [P, C.c_int] + [vp] * 13 + [sz, vp]
+        L.ra_attn_int4_s8.argtypes = [P] + [vp] * 9
         L.ra_sync_status.argtypes = [vp]
         for name in ("ra_rope_rotate_quant", "ra_attn_int4", "ra_test_int4_codes", "ra_rope_bf16",
                      "ra_attn_bf16_fallback", "ra_sync_status", "ra_attn_int4_opts", "ra_test_int4_codes_opts",
-                     "ra_attn_int4_qfused"):
+                     "ra_attn_int4_qfused", "ra_rope_rotate_quant_s8", "ra_attn_int4_s8"):
             getattr(L, name).restype = C.c_int
         _lib = L
     return _lib
@@ -186,6 +188,58 @@ def attn_int4(p: Problem, codes: Dict[str, torch.Tensor], out: Optional[torch.Te
         _ptr(out, torch.bfloat16, (B, H, N, D), "out"), _ptr(lse, torch.float32, (B, H, N), "lse"),
         C.c_void_p(_stream(stream)))
     _check("ra_attn_int4_opts", rc)
+    return out
+
+
+def rope_rotate_quant_s8(p: Problem, q: Optional[torch.Tensor], k: torch.Tensor, v: torch.Tensor,
+                         pos: torch.Tensor, out: Optional[Dict[str, torch.Tensor]] = None,
+                         workspace: Optional[torch.Tensor] = None, stream=None) -> Dict[str, torch.Tensor]:
+    """ra_rope_rotate_quant_s8: returns q8, sq, k8, sk, k_mean, v8, sv, v_colsum, the
+    codes as int8 16 x code [B, H, N, D] (q = None: K and V only)."""
+    B, H, N, D = p.B, p.H, p.N, p.D
+    dev = k.device
+    if out is None:
+        out = {} if q is None else {
+            "q8": torch.empty(B, H, N, D, dtype=torch.int8, device=dev),
+            "sq": torch.empty(B, H, N, dtype=torch.float32, device=dev)}
+        out.update({
+            "k8": torch.empty(B, H, N, D, dtype=torch.int8, device=dev),
+            "sk": torch.empty(B, H, N, dtype=torch.float32, device=dev),
+            "k_mean": torch.empty(B, H, D, dtype=torch.float32, device=dev),
+            "v8": torch.empty(B, H, N, D, dtype=torch.int8, device=dev),
+            "sv": torch.empty(B, H, D, dtype=torch.float32, device=dev),
+            "v_colsum": torch.empty(B, H, _nblocks(p), D, dtype=torch.int32, device=dev),
+        })
+    if workspace is None:
+        workspace = torch.empty(max(workspace_bytes(p), 16), dtype=torch.uint8, device=dev)
+    shp = (B, H, N, D)
+    rc = lib().ra_rope_rotate_quant_s8(
+        C.byref(p), _in_dtype(k), _ptr(q, k.dtype, shp, "q"), _ptr(k, k.dtype, shp, "k"), _ptr(v, k.dtype, shp, "v"),
+        _ptr(pos, torch.int32, (N, 3), "pos"),
+        _ptr(out.get("q8") if q is not None else None, torch.int8, shp),
+        _ptr(out.get("sq") if q is not None else None, torch.float32, (B, H, N)),
+        _ptr(out["k8"], torch.int8, shp), _ptr(out["sk"], torch.float32, (B, H, N)),
+        _ptr(out["k_mean"], torch.float32, (B, H, D)), _ptr(out["v8"], torch.int8, shp),
+        _ptr(out["sv"], torch.float32, (B, H, D)), _ptr(out["v_colsum"], torch.int32, (B, H, _nblocks(p), D)),
+        _ptr(workspace, torch.uint8), C.c_size_t(workspace.numel()), C.c_void_p(_stream(stream)))
+    _check("ra_rope_rotate_quant_s8", rc)
+    return out
+
+
+def attn_int4_s8(p: Problem, codes: Dict[str, torch.Tensor], out: Optional[torch.Tensor] = None,
+                 lse: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """ra_attn_int4_s8 on rope_rotate_quant_s8's outputs; returns out [B, H, N, D] bf16."""
+    B, H, N, D = p.B, p.H, p.N, p.D
+    shp = (B, H, N, D)
+    if out is None:
+        out = torch.empty(shp, dtype=torch.bfloat16, device=codes["q8"].device)
+    rc = lib().ra_attn_int4_s8(
+        C.byref(p), _ptr(codes["q8"], torch.int8, shp), _ptr(codes["sq"], torch.float32, (B, H, N)),
+        _ptr(codes["k8"], torch.int8, shp), _ptr(codes["sk"], torch.float32, (B, H, N)),
+        _ptr(codes["v8"], torch.int8, shp), _ptr(codes["sv"], torch.float32, (B, H, D)),
+        _ptr(out, torch.bfloat16, shp, "out"), _ptr(lse, torch.float32, (B, H, N), "lse"),
+        C.c_void_p(_stream(stream)))
+    _check("ra_attn_int4_s8", rc)
     return out
 
 

@@ -259,13 +259,17 @@ __device__ __forceinline__ bool wait_at(uint64_t* bar, uint32_t parity, volatile
 
 // MODE bits 0-1: P codes (0 range-rectified, 1 block-local maximum, 2
 // symmetric); bit 2: fp32 denominator; bit 3: fused Q (warp 3 computes Q's
-// packed codes and scales from the raw Q in place of the TMA load of q4).
+// packed codes and scales from the raw Q in place of the TMA load of q4);
+// bit 4: s8 code layout (one code per byte as 16 x code, natural channel
+// order): the TMA loads Q, K and V straight into the MMA operand tiles, and
+// warps 4-7 only stage the per-key scales.
 template <int D, int BN, bool DUMP, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                  const __grid_constant__ CUtensorMap tm_v, const AttnParams prm) {
   using C = Cfg<D, BN>;
   constexpr bool kFQ = (MODE & 8) != 0;
+  constexpr bool kS8 = (MODE & 16) != 0;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte aligned base; pointer arithmetic on the shared array keeps the
   // shared address space visible to the compiler (LDS/STS, not generic LD/ST).
@@ -286,10 +290,12 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    mbar_init(B.qpk_full, 1); mbar_init(B.qpk_empty, 4); mbar_init(B.q_full, 4); mbar_init(B.q_free, 2);
+    // s8 layout: the TMA fills Q, K and V tiles (one expect-tx arrival each);
+    // a K stage also waits for the four scale warps.
+    mbar_init(B.qpk_full, 1); mbar_init(B.qpk_empty, 4); mbar_init(B.q_full, kS8 ? 1 : 4); mbar_init(B.q_free, 2);
     for (int s = 0; s < C::kPS; ++s) { mbar_init(B.pk_full + s, 1); mbar_init(B.pk_empty + s, 4); }
-    for (int s = 0; s < C::kKS; ++s) { mbar_init(B.kw_full + s, 4); mbar_init(B.kw_empty + s, 2 + 16); }
-    for (int s = 0; s < C::kVS; ++s) { mbar_init(B.vw_full + s, 4); mbar_init(B.vw_empty + s, 2); }
+    for (int s = 0; s < C::kKS; ++s) { mbar_init(B.kw_full + s, kS8 ? 1 + 4 : 4); mbar_init(B.kw_empty + s, 2 + 16); }
+    for (int s = 0; s < C::kVS; ++s) { mbar_init(B.vw_full + s, kS8 ? 1 : 4); mbar_init(B.vw_empty + s, 2); }
     for (int s = 0; s < 4; ++s) { mbar_init(B.s_full + s, 1); mbar_init(B.p_full + s, 8); mbar_init(B.pv_done + s, 1); }
     mbar_init(B.drain, 1);
     mbar_init(B.drain + 1, 1);
@@ -319,7 +325,37 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     else asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
     if (warp == 0) {
       // ------------------------------------------------------------ TMA producer
-      if (lane == 0) {
+      if (kS8 && lane == 0) {
+        // s8 layout: K and V of each block into their operand stages, and the
+        // item's Q tiles after its first block (once the previous item's QK
+        // products have been issued).
+        uint32_t g = 0, li = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; item < prm.nitems && ok; item += gridDim.x, ++li) {
+          const int bh = item / prm.npairs, pair = item % prm.npairs;
+          for (int t = 0; t < nb; ++t, ++g) {
+            const int ks = g % C::kKS, vs = g % C::kVS;
+            if (!(ok = wait_at(B.kw_empty + ks, ((g / C::kKS) & 1) ^ 1, abort_flag, 14u, g, 256u))) break;
+            mbar_arrive_expect_tx(B.kw_full + ks, C::kKwBytes);
+            tma_load_3d(smem + C::oKw + ks * C::kKwStride, &tm_k, B.kw_full + ks, 0, t * BN, bh);
+            if (!(ok = wait_at(B.vw_empty + vs, ((g / C::kVS) & 1) ^ 1, abort_flag, 16u, g, 256u))) break;
+            mbar_arrive_expect_tx(B.vw_full + vs, C::kVwBytes);
+            tma_load_3d(smem + C::oVw + vs * C::kVwStride, &tm_v, B.vw_full + vs, 0, t * BN, bh);
+            if (t == 0) {
+              if (!(ok = wait_at(B.q_free, (li & 1) ^ 1, abort_flag, 1u, li, 256u))) break;
+              mbar_arrive_expect_tx(B.q_full, kTiles * C::kQBytes);
+              for (int tt = 0; tt < kTiles; ++tt)
+                tma_load_3d(smem + C::oQ + tt * C::kQBytes, &tm_q, B.q_full, 0, pair * 2 * kRows + tt * kRows, bh);
+            }
+          }
+        }
+        // Wait (bounded) for the copies of the last stages to land.
+        for (uint32_t k = (g > (uint32_t)C::kKS ? g - C::kKS : 0); k < g; ++k) {
+          uint32_t it = 0;
+          while (!mbar_try_wait(B.vw_full + (k % C::kVS), (k / C::kVS) & 1) && ++it < kSpinLimit) {}
+        }
+        if (!ok) set_status(kStatusTimeout);
+      } else if (!kS8 && lane == 0) {
         uint32_t g = 0, li = 0;
         bool ok = true;
         for (int item = blockIdx.x; item < prm.nitems && ok; item += gridDim.x, ++li) {
@@ -436,6 +472,29 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
         if (!ok) set_status(kStatusTimeout);
       }
+    } else if (warp >= 4 && kS8) {
+      // ------------------------------------------------------------ scale warps (s8 layout)
+      // The TMA fills the operand tiles; these warps only stage each block's
+      // per-key scales (the K stage's barrier waits for them too).
+      const int wt = threadIdx.x - 128;  // 0..127
+      uint32_t g = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < prm.nitems && ok; item += gridDim.x) {
+        const int bh = item / prm.npairs;
+        for (int t = 0; t < nb; ++t, ++g) {
+          const int ks = g % C::kKS;
+          if (!(ok = wait_at(B.kw_empty + ks, ((g / C::kKS) & 1) ^ 1, abort_flag, 15u, g, 256u))) break;
+          if (wt < BN) {
+            const int j = t * BN + wt;
+            float* ksc = reinterpret_cast<float*>(smem + C::oKsc) + ks * BN;
+            ksc[wt] = j < prm.N ? prm.sk[static_cast<size_t>(bh) * prm.N + j] * (1.0f / 256.0f)
+                                : __int_as_float(0x7FC00000);
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(B.kw_full + ks);
+        }
+      }
+      if (!ok) set_status(kStatusTimeout);
     } else if (warp >= 4) {
       // ------------------------------------------------------------ widening warps
       const int wt = threadIdx.x - 128;  // 0..127
@@ -772,7 +831,8 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           return i < kFr ? ((i & 1) ? F2[i >> 1].y : F2[i >> 1].x) : Fsf[i - kFr];
         };
         // Widened positions hh * D/2 + c + (4a + b) and + 16 hold channels
-        // d = hh * D/2 + c + 8a + 2b and d + 1.
+        // d = hh * D/2 + c + 8a + 2b and d + 1 (packed layout); in the s8
+        // layout position p is channel p.
 #pragma unroll
         for (int c = 0; c < kHD; c += 32) {
           const int c0 = hh * kHD + c;
@@ -781,9 +841,9 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           for (int a = 0; a < 4; ++a)
 #pragma unroll
             for (int b = 0; b < 4; ++b) {
-              const int d = c0 + 8 * a + 2 * b;
-              const float f0 = fget(c + 4 * a + b);
-              const float f1 = fget(c + 16 + 4 * a + b);
+              const int d = kS8 ? c0 + 2 * (4 * a + b) : c0 + 8 * a + 2 * b;
+              const float f0 = kS8 ? fget(c + 2 * (4 * a + b)) : fget(c + 4 * a + b);
+              const float f1 = kS8 ? fget(c + 2 * (4 * a + b) + 1) : fget(c + 16 + 4 * a + b);
               const __nv_bfloat162 h2 = __floats2bfloat162_rn(f0 * __ldg(sv + d) * inv, f1 * __ldg(sv + d + 1) * inv);
               pk[4 * a + b] = *reinterpret_cast<const uint32_t*>(&h2);
             }
@@ -831,15 +891,35 @@ bool make_code_map(CUtensorMap* m, const void* base, int BH, int N, int D, int r
   return r == CUDA_SUCCESS;
 }
 
+// 3D map over s8 codes [BH, N, D] bytes; box = rows x D, swizzled like the
+// widened operand tiles (128B for D = 128, 64B for D = 64); zero fill past N.
+bool make_s8_map(CUtensorMap* m, const void* base, int BH, int N, int D, int rows) {
+  auto enc = get_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N) * D};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(D), static_cast<cuuint32_t>(rows), 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 template <int D, int BN, bool DUMP, int MODE>
 cudaError_t launch_cfg(const ra_problem& p, const uint8_t* q4, const uint8_t* k4, const uint8_t* v4,
                        const AttnParams& prm, cudaStream_t st) {
   using C = Cfg<D, BN>;
   CUtensorMap mq, mk, mv;
   const int BH = p.B * p.H;
-  if (!make_code_map(&mq, q4, BH, p.N, D, kRows) || !make_code_map(&mk, k4, BH, p.N, D, BN) ||
-      !make_code_map(&mv, v4, BH, p.N, D, BN))
+  if constexpr ((MODE & 16) != 0) {
+    if (!make_s8_map(&mq, q4, BH, p.N, D, kRows) || !make_s8_map(&mk, k4, BH, p.N, D, BN) ||
+        !make_s8_map(&mv, v4, BH, p.N, D, BN))
+      return cudaErrorInvalidValue;
+  } else if (!make_code_map(&mq, q4, BH, p.N, D, kRows) || !make_code_map(&mk, k4, BH, p.N, D, BN) ||
+             !make_code_map(&mv, v4, BH, p.N, D, BN)) {
     return cudaErrorInvalidValue;
+  }
   auto kern = attn_int4_kernel<D, BN, DUMP, MODE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
@@ -884,6 +964,15 @@ cudaError_t launch_attn_int4(const ra_problem& p, const uint8_t* q4, const float
     prm.rot = p.rot; prm.seg = seg_info(p);
     return p.D == 128 ? launch_cfg<128, 64, false, 8>(p, k4, k4, v4, prm, st)
                       : launch_cfg<64, 64, false, 8>(p, k4, k4, v4, prm, st);
+  }
+  if (mode == 16) {
+    // s8 code layout: block_k = 64, the method's P codes and denominator, no dump.
+    if (p.block_k != 64 || dmp) {
+      *unsupported = 1;
+      return cudaSuccess;
+    }
+    return p.D == 128 ? launch_cfg<128, 64, false, 16>(p, q4, k4, v4, prm, st)
+                      : launch_cfg<64, 64, false, 16>(p, q4, k4, v4, prm, st);
   }
   if (p.block_k == 128)
     return launch_attn_int4_pair(p, q4, sq, k4, sk, v4, sv, out, lse, dump, mode, st, unsupported);

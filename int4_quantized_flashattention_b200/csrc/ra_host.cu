@@ -58,10 +58,32 @@ size_t ra_workspace_bytes(const ra_problem* p) {
   return ra::workspace_layout(*p).total;
 }
 
+static ra_status rope_rotate_quant(const ra_problem* p, int in_dtype, const void* q, const void* k,
+                                   const void* v, const int32_t* pos, uint8_t* q4, float* sq, uint8_t* k4,
+                                   float* sk, float* k_mean, uint8_t* v4, float* sv, int32_t* v_colsum,
+                                   void* workspace, size_t ws_bytes, void* stream, bool s8);
+
 ra_status ra_rope_rotate_quant(const ra_problem* p, int in_dtype, const void* q, const void* k,
                                const void* v, const int32_t* pos, uint8_t* q4, float* sq, uint8_t* k4,
                                float* sk, float* k_mean, uint8_t* v4, float* sv, int32_t* v_colsum,
                                void* workspace, size_t ws_bytes, void* stream) {
+  return rope_rotate_quant(p, in_dtype, q, k, v, pos, q4, sq, k4, sk, k_mean, v4, sv, v_colsum, workspace,
+                           ws_bytes, stream, false);
+}
+
+ra_status ra_rope_rotate_quant_s8(const ra_problem* p, int in_dtype, const void* q, const void* k,
+                                  const void* v, const int32_t* pos, int8_t* q8, float* sq, int8_t* k8,
+                                  float* sk, float* k_mean, int8_t* v8, float* sv, int32_t* v_colsum,
+                                  void* workspace, size_t ws_bytes, void* stream) {
+  return rope_rotate_quant(p, in_dtype, q, k, v, pos, reinterpret_cast<uint8_t*>(q8), sq,
+                           reinterpret_cast<uint8_t*>(k8), sk, k_mean, reinterpret_cast<uint8_t*>(v8), sv, v_colsum,
+                           workspace, ws_bytes, stream, true);
+}
+
+static ra_status rope_rotate_quant(const ra_problem* p, int in_dtype, const void* q, const void* k,
+                                   const void* v, const int32_t* pos, uint8_t* q4, float* sq, uint8_t* k4,
+                                   float* sk, float* k_mean, uint8_t* v4, float* sv, int32_t* v_colsum,
+                                   void* workspace, size_t ws_bytes, void* stream, bool s8) {
   if (!valid_problem(p) || (in_dtype != RA_DT_F32 && in_dtype != RA_DT_BF16)) return RA_ERR_INVALID_ARG;
   // Q, q4 and sq are either all given or all NULL (K and V only).
   const bool no_q = !q && !q4 && !sq;
@@ -71,7 +93,25 @@ ra_status ra_rope_rotate_quant(const ra_problem* p, int in_dtype, const void* q,
   if (!no_q && (!aligned16(q) || !aligned16(q4) || !aligned16(sq))) return RA_ERR_INVALID_ARG;
   if (ws_bytes < ra::workspace_layout(*p).total) return RA_ERR_INVALID_ARG;
   return from_cuda(ra::launch_prologue(*p, in_dtype, q, k, v, pos, q4, sq, k4, sk, k_mean, v4, sv, v_colsum,
-                                       workspace, static_cast<cudaStream_t>(stream)));
+                                       workspace, static_cast<cudaStream_t>(stream), s8));
+}
+
+ra_status ra_attn_int4_s8(const ra_problem* p, const int8_t* q8, const float* sq, const int8_t* k8,
+                          const float* sk, const int8_t* v8, const float* sv, void* out, float* lse,
+                          void* stream) {
+  if (!valid_problem(p)) return RA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q8, sq, k8, sk, v8, sv, out};
+  for (const void* x : ptrs)
+    if (!aligned16(x)) return RA_ERR_INVALID_ARG;
+  if (!aligned16_or_null(lse)) return RA_ERR_INVALID_ARG;
+  if (p->block_k != 64) return RA_ERR_UNSUPPORTED;
+  int unsupported = 0;
+  cudaError_t e = ra::launch_attn_int4(*p, reinterpret_cast<const uint8_t*>(q8), sq,
+                                       reinterpret_cast<const uint8_t*>(k8), sk,
+                                       reinterpret_cast<const uint8_t*>(v8), sv, out, lse, nullptr, 16,
+                                       static_cast<cudaStream_t>(stream), &unsupported);
+  if (unsupported) return RA_ERR_UNSUPPORTED;
+  return from_cuda(e);
 }
 
 ra_status ra_attn_int4_qfused(const ra_problem* p, int in_dtype, const void* q, const int32_t* pos,

@@ -21,7 +21,7 @@ WorkspaceLayout workspace_layout(const ra_problem& p);
 cudaError_t launch_prologue(const ra_problem& p, int dtype, const void* q, const void* k, const void* v,
                             const int32_t* pos, uint8_t* q4, float* sq, uint8_t* k4, float* sk,
                             float* k_mean, uint8_t* v4, float* sv, int32_t* colsum, void* ws,
-                            cudaStream_t st);
+                            cudaStream_t st, bool s8 = false);
 cudaError_t launch_rope_bf16(const ra_problem& p, int dtype, const void* q, const void* k,
                              const int32_t* pos, void* qo, void* ko, void* ws, cudaStream_t st);
 cudaError_t read_prologue_status(uint32_t* out);

@@ -97,9 +97,10 @@ struct PrologueArgs {
   double* ksum;     // [BH, nchunk, D]
   float* vmax;      // [BH, nchunk, D]
   float* vinv;      // [BH, D]
-  uint8_t *q4, *k4, *v4;
+  uint8_t *q4, *k4, *v4;   // packed codes [BH, N, D/2], or s8 codes [BH, N, D] when s8
   float *sq, *sk, *k_mean, *sv;
   int32_t* colsum;
+  int s8;                  // code layout: 0 packed nibbles, 1 one code per byte (16 x code)
 };
 
 // Table entry e -> (segment j, position g, pair k); angle g * theta^(-2k/Dj) in
@@ -329,7 +330,7 @@ __global__ void prologue_finalize_kernel(PrologueArgs a) {
 // one key block, then combined across the warp's tokens and added to shared
 // memory.  kQ = false leaves Q out (the attention kernel's fused-Q path
 // quantises Q itself): only K and V are staged and written.
-template <bool kBf16, int kRot, int kD, bool kQ>
+template <bool kBf16, int kRot, int kD, bool kQ, bool kS8>
 __global__ void __launch_bounds__(kThreads, 3) prologue_quant_kernel(PrologueArgs a) {
   constexpr int kNT = kQ ? 3 : 2;          // staged tensors
   constexpr int iK = kQ ? 1 : 0, iV = iK + 1;
@@ -441,9 +442,16 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_quant_kernel(PrologueArg
       }
       if (valid) {
         const size_t o4 = head4 + static_cast<size_t>(n) * (kD / 2) + (c0 >> 1);
-        if constexpr (kQ) *reinterpret_cast<uint32_t*>(a.q4 + o4) = pack8_bits(bq);
-        *reinterpret_cast<uint32_t*>(a.k4 + o4) = pack8_bits(bk);
-        *reinterpret_cast<uint32_t*>(a.v4 + o4) = pack8_bits(bv);
+        if constexpr (kS8) {
+          const size_t o8 = head + static_cast<size_t>(n) * kD + c0;
+          if constexpr (kQ) *reinterpret_cast<uint2*>(a.q4 + o8) = make_uint2(pack4_s8_bits(bq), pack4_s8_bits(bq + 4));
+          *reinterpret_cast<uint2*>(a.k4 + o8) = make_uint2(pack4_s8_bits(bk), pack4_s8_bits(bk + 4));
+          *reinterpret_cast<uint2*>(a.v4 + o8) = make_uint2(pack4_s8_bits(bv), pack4_s8_bits(bv + 4));
+        } else {
+          if constexpr (kQ) *reinterpret_cast<uint32_t*>(a.q4 + o4) = pack8_bits(bq);
+          *reinterpret_cast<uint32_t*>(a.k4 + o4) = pack8_bits(bk);
+          *reinterpret_cast<uint32_t*>(a.v4 + o4) = pack8_bits(bv);
+        }
         if (c0 == 0) {
           if constexpr (kQ) a.sq[static_cast<size_t>(bh) * a.N + n] = __fdiv_rn(mq, 7.0f);
           a.sk[static_cast<size_t>(bh) * a.N + n] = __fdiv_rn(mk, 7.0f);
@@ -552,6 +560,21 @@ static cudaError_t launch_tables(const ra_problem& p, int rot, float2* tab, cuda
   return cudaGetLastError();
 }
 
+// The quantise pass, with or without Q, in one code layout.
+template <bool kBf16, int kRot, int kD, bool kS8>
+static cudaError_t launch_quant(const PrologueArgs& a, dim3 grid, int quant_bytes, cudaStream_t st) {
+  cudaError_t e;
+  if (a.q) {
+    if ((e = set_smem(prologue_quant_kernel<kBf16, kRot, kD, true, kS8>, quant_bytes)) != cudaSuccess) return e;
+    prologue_quant_kernel<kBf16, kRot, kD, true, kS8><<<grid, kThreads, quant_bytes, st>>>(a);
+  } else {
+    const int kv_bytes = quant_bytes / 3 * 2;
+    if ((e = set_smem(prologue_quant_kernel<kBf16, kRot, kD, false, kS8>, kv_bytes)) != cudaSuccess) return e;
+    prologue_quant_kernel<kBf16, kRot, kD, false, kS8><<<grid, kThreads, kv_bytes, st>>>(a);
+  }
+  return cudaGetLastError();
+}
+
 // The three passes (channel reduce, finalize, quantise) for one input type and
 // rotation mode and head dimension.
 template <bool kBf16, int kRot, int kD>
@@ -563,15 +586,8 @@ static cudaError_t launch_passes3(const PrologueArgs& a, dim3 grid, int red_byte
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   prologue_finalize_kernel<<<grid.y, 128, 0, st>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if (a.q) {
-    if ((e = set_smem(prologue_quant_kernel<kBf16, kRot, kD, true>, quant_bytes)) != cudaSuccess) return e;
-    prologue_quant_kernel<kBf16, kRot, kD, true><<<grid, kThreads, quant_bytes, st>>>(a);
-  } else {
-    const int kv_bytes = quant_bytes / 3 * 2;
-    if ((e = set_smem(prologue_quant_kernel<kBf16, kRot, kD, false>, kv_bytes)) != cudaSuccess) return e;
-    prologue_quant_kernel<kBf16, kRot, kD, false><<<grid, kThreads, kv_bytes, st>>>(a);
-  }
-  return cudaGetLastError();
+  if (a.s8) return launch_quant<kBf16, kRot, kD, true>(a, grid, quant_bytes, st);
+  return launch_quant<kBf16, kRot, kD, false>(a, grid, quant_bytes, st);
 }
 
 template <bool kBf16, int kRot>
@@ -584,7 +600,7 @@ static cudaError_t launch_passes(const PrologueArgs& a, dim3 grid, int red_bytes
 cudaError_t launch_prologue(const ra_problem& p, int dtype, const void* q, const void* k, const void* v,
                             const int32_t* pos, uint8_t* q4, float* sq, uint8_t* k4, float* sk,
                             float* k_mean, uint8_t* v4, float* sv, int32_t* colsum, void* ws,
-                            cudaStream_t st) {
+                            cudaStream_t st, bool s8) {
   const WorkspaceLayout w = workspace_layout(p);
   char* base = static_cast<char*>(ws);
   PrologueArgs a;
@@ -600,6 +616,7 @@ cudaError_t launch_prologue(const ra_problem& p, int dtype, const void* q, const
   a.vinv = reinterpret_cast<float*>(base + w.vinv);
   a.q4 = q4; a.k4 = k4; a.v4 = v4; a.sq = sq; a.sk = sk; a.k_mean = k_mean; a.sv = sv;
   a.colsum = colsum;
+  a.s8 = s8 ? 1 : 0;
   cudaError_t e = launch_tables(p, p.rot, reinterpret_cast<float2*>(base + w.tab), st);
   if (e != cudaSuccess) return e;
   if (p.rot == 1) {  // the fused table differs from the plain one

@@ -238,6 +238,21 @@ __device__ __forceinline__ uint32_t pack8_bits(const uint32_t* b) {
   return (acc - kQBitsRep) ^ 0x88888888u;
 }
 
+// The s8 code layout: one code per byte, held in the byte's high nibble (the
+// s8 value 16 x code, the low nibble zero), channels in natural order.  For
+// four quant4_bits2 results b[0..3] (channels c..c+3) the little-endian word
+// of their bytes: sum_i 256^i b_i minus the known offsets leaves the bytes
+// code + 8 (at most 15: no carries), shifted into the high nibble; XOR 0x80
+// turns (code + 8) * 16 into the s8 value 16 x code.
+constexpr uint32_t kQBitsRep4 = kQBits * 0x01010101u;   // sum_i 256^i 0x4B400000 mod 2^32
+__device__ __forceinline__ uint32_t pack4_s8_bits(const uint32_t* b) {
+  uint32_t acc = b[3];
+  acc = acc * 256u + b[2];
+  acc = acc * 256u + b[1];
+  acc = acc * 256u + b[0];
+  return ((acc - kQBitsRep4) << 4) ^ 0x80808080u;
+}
+
 // Max over the D/8 threads of a token (a contiguous lane group of size lpt).
 __device__ __forceinline__ float group_max(float v, int lpt) {
   for (int o = lpt >> 1; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));

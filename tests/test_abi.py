@@ -37,7 +37,8 @@ def test_header_declares_the_entry_points():
     names = _declared()
     for n in ("ra_rope_rotate_quant", "ra_attn_int4", "ra_attn_bf16_fallback", "ra_test_int4_codes",
               "ra_rope_bf16", "ra_workspace_bytes", "ra_sync_status", "ra_status_string",
-              "ra_attn_int4_opts", "ra_test_int4_codes_opts", "ra_attn_int4_qfused"):
+              "ra_attn_int4_opts", "ra_test_int4_codes_opts", "ra_attn_int4_qfused",
+              "ra_rope_rotate_quant_s8", "ra_attn_int4_s8"):
         assert n in names
 
 
@@ -201,3 +202,24 @@ def test_kv_only_prologue_needs_all_three_q_pointers_null(ra):
     for i in (0, 4, 5):
         args[i] = None
     assert L.ra_rope_rotate_quant(C.byref(p), 1, *args, need, None) not in (1, 2)
+
+
+def test_s8_entries_validate_before_any_launch(ra):
+    """ra_attn_int4_s8 / ra_rope_rotate_quant_s8: bad arguments are
+    RA_ERR_INVALID_ARG and block sizes other than 64 RA_ERR_UNSUPPORTED before
+    any launch (no GPU needed)."""
+    L = ra.lib()
+    good, bad = C.c_void_p(0x10000), C.c_void_p(0x10004)
+    p = _wan(ra)
+    for i in range(7):
+        args = [good] * 7
+        args[i] = bad
+        assert L.ra_attn_int4_s8(C.byref(p), *args, None, None) == 1
+        args[i] = None
+        assert L.ra_attn_int4_s8(C.byref(p), *args, None, None) == 1
+    assert L.ra_attn_int4_s8(C.byref(p), *([good] * 7), bad, None) == 1
+    assert L.ra_attn_int4_s8(C.byref(_wan(ra, block_k=32)), *([good] * 7), None, None) == 2
+    assert L.ra_attn_int4_s8(C.byref(_wan(ra, block_k=128)), *([good] * 7), None, None) == 2
+    need = ra.workspace_bytes(p)
+    assert L.ra_rope_rotate_quant_s8(C.byref(p), 1, *([good] * 13), C.c_size_t(need - 16), None) == 1
+    assert L.ra_rope_rotate_quant_s8(C.byref(p), 7, *([good] * 13), C.c_size_t(need), None) == 1

@@ -1,0 +1,73 @@
+"""The s8 code layout (ra_rope_rotate_quant_s8 / ra_attn_int4_s8): one code
+per byte as 16 x code, natural channel order, loaded by TMA straight into the
+MMA operand tiles.  The codes must be the packed prologue's codes (times 16)
+bit for bit, every other prologue output identical, and the attention's out
+and lse identical to ra_attn_int4 on the packed codes; the packed path is
+checked against the oracle in test_gpu_int4.py.
+"""
+import numpy as np
+import pytest
+
+from synth import inputs as si
+from tests import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def ra():
+    import __graft_entry__
+    __graft_entry__.build()
+    import int4_quantized_flashattention_b200 as ra
+    return ra
+
+
+def _unpack16(packed):
+    import oracle
+    return (oracle.unpack_codes(packed).astype(np.int16) * 16).astype(np.int8)
+
+
+def _run(ra, wl):
+    import torch
+    dev = gu.device()
+    x = si.make_inputs(wl)
+    p = gu.problem_for(ra, wl)
+    q, k, v, pos = gu.to_device(x, wl, dev)
+    packed = ra.rope_rotate_quant(p, q, k, v, pos)
+    lse_ref = torch.empty(wl.B, wl.H, wl.N, dtype=torch.float32, device=dev)
+    out_ref = ra.attn_int4(p, packed, lse=lse_ref)
+    assert ra.sync_status() == 0
+    s8 = ra.rope_rotate_quant_s8(p, q, k, v, pos)
+    assert ra.sync_status() == 0
+    for a, b in (("q8", "q4"), ("k8", "k4"), ("v8", "v4")):
+        got = s8[a].cpu().numpy().reshape(-1, wl.D)
+        ref = _unpack16(packed[b].cpu().numpy().reshape(-1, wl.D // 2))
+        assert np.array_equal(got, ref), a
+    for name in ("sq", "sk", "k_mean", "sv", "v_colsum"):
+        assert torch.equal(s8[name], packed[name]), name
+    out = torch.full_like(out_ref, float("nan"))
+    lse = torch.full_like(lse_ref, float("nan"))
+    ra.attn_int4_s8(p, s8, out=out, lse=lse)
+    assert ra.sync_status() == 0
+    assert torch.equal(out.view(torch.int16), out_ref.view(torch.int16))
+    assert torch.equal(lse.view(torch.int32), lse_ref.view(torch.int32))
+
+
+@pytest.mark.parametrize("D,seg,rot,grid", [
+    (128, (44, 42, 42), 1, (3, 10, 10)),   # N = 300: ragged query tile and key block
+    (128, (16, 56, 56), 2, (2, 5, 9)),     # N = 90: one partial block
+    (64, (24, 20, 20), 1, (5, 9, 11)),     # D = 64, N = 495
+    (64, (24, 20, 20), 0, (1, 1, 7)),      # N = 7
+    (128, (44, 42, 42), 3, (1, 1, 1)),     # N = 1
+])
+def test_s8_equals_packed(ra, D, seg, rot, grid):
+    wl = si.WORKLOADS["small"].with_(H=2, D=D, seg=seg, grid=grid, rot=rot, block_k=64)
+    _run(ra, wl)
+
+
+def test_s8_at_the_wan_shape(ra):
+    _run(ra, si.WORKLOADS["wan"])
+
+
+def test_s8_sharp(ra):
+    _run(ra, si.WORKLOADS["small"].with_(H=2, sharp=True))
