@@ -144,28 +144,32 @@ ra_status ra_attn_int4(const ra_problem* p,
                        void* out, float* lse, void* stream);
 
 /*
- * The s8 code layout: the same codes with one code per byte, held in the
- * byte's high nibble (the int8 value 16 x code, low nibble zero), channels in
- * natural order: [B, H, N, D] int8.  On sm_100a the tensor cores have no 4-bit
- * integer kind, so packed nibbles must be widened to bytes before every MMA;
- * in this layout the attention kernel loads Q, K and V tiles by TMA straight
- * into its MMA operands and skips the widening (twice the code bytes in HBM).
- * ra_rope_rotate_quant_s8 takes the arguments of ra_rope_rotate_quant (q, q8,
- * sq may be NULL together) and writes q8, k8, v8 in this layout; every other
- * output is identical.  ra_attn_int4_s8 takes the arguments of ra_attn_int4
- * with the s8 codes; its out and lse equal ra_attn_int4's on the packed codes
- * bit for bit.  Implemented for block_k = 64 (D = 64 or 128), the method's P
- * codes and denominator; other block sizes return RA_ERR_UNSUPPORTED.
+ * The byte code layout: the same INT4 codes with one code per byte, channels
+ * in natural order, [B, H, N, D] bytes: q8 and k8 hold the FP8 E4M3 value
+ * equal to the code (every integer in [-7, 7] is exact in E4M3), v8 the int8
+ * value 16 x code (the code in the high nibble).  On sm_100a the tensor cores
+ * have no 4-bit integer kind, so packed nibbles must be widened to bytes
+ * before every MMA; in this layout the attention kernel loads Q, K and V tiles
+ * by TMA straight into its MMA operands and skips the widening (twice the code
+ * bytes in HBM), and Q K^T runs as an FP8 MMA with an fp32 accumulator, which
+ * is exact here (|S_int| <= 49 D < 2^13) and spares the softmax its integer
+ * conversion.  ra_rope_rotate_quant_s8 takes the arguments of
+ * ra_rope_rotate_quant (q, q8, sq may be NULL together) and writes q8, k8, v8
+ * in this layout; every other output is identical.  ra_attn_int4_s8 takes the
+ * arguments of ra_attn_int4 with these codes; its out and lse equal
+ * ra_attn_int4's on the packed codes bit for bit.  Implemented for
+ * block_k = 64 (D = 64 or 128), the method's P codes and denominator; other
+ * block sizes return RA_ERR_UNSUPPORTED.
  */
 ra_status ra_rope_rotate_quant_s8(const ra_problem* p, int in_dtype,
                                   const void* q, const void* k, const void* v,
                                   const int32_t* pos,
-                                  int8_t* q8, float* sq, int8_t* k8, float* sk,
+                                  uint8_t* q8, float* sq, uint8_t* k8, float* sk,
                                   float* k_mean, int8_t* v8, float* sv, int32_t* v_colsum,
                                   void* workspace, size_t ws_bytes, void* stream);
 ra_status ra_attn_int4_s8(const ra_problem* p,
-                          const int8_t* q8, const float* sq,
-                          const int8_t* k8, const float* sk,
+                          const uint8_t* q8, const float* sq,
+                          const uint8_t* k8, const float* sk,
                           const int8_t* v8, const float* sv,
                           void* out, float* lse, void* stream);
 

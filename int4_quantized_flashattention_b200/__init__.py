@@ -194,16 +194,17 @@ def attn_int4(p: Problem, codes: Dict[str, torch.Tensor], out: Optional[torch.Te
 def rope_rotate_quant_s8(p: Problem, q: Optional[torch.Tensor], k: torch.Tensor, v: torch.Tensor,
                          pos: torch.Tensor, out: Optional[Dict[str, torch.Tensor]] = None,
                          workspace: Optional[torch.Tensor] = None, stream=None) -> Dict[str, torch.Tensor]:
-    """ra_rope_rotate_quant_s8: returns q8, sq, k8, sk, k_mean, v8, sv, v_colsum, the
-    codes as int8 16 x code [B, H, N, D] (q = None: K and V only)."""
+    """ra_rope_rotate_quant_s8: returns q8, sq, k8, sk, k_mean, v8, sv, v_colsum with
+    the codes one per byte [B, H, N, D]: q8, k8 FP8 E4M3 bytes (uint8 tensors),
+    v8 int8 16 x code (q = None: K and V only)."""
     B, H, N, D = p.B, p.H, p.N, p.D
     dev = k.device
     if out is None:
         out = {} if q is None else {
-            "q8": torch.empty(B, H, N, D, dtype=torch.int8, device=dev),
+            "q8": torch.empty(B, H, N, D, dtype=torch.uint8, device=dev),
             "sq": torch.empty(B, H, N, dtype=torch.float32, device=dev)}
         out.update({
-            "k8": torch.empty(B, H, N, D, dtype=torch.int8, device=dev),
+            "k8": torch.empty(B, H, N, D, dtype=torch.uint8, device=dev),
             "sk": torch.empty(B, H, N, dtype=torch.float32, device=dev),
             "k_mean": torch.empty(B, H, D, dtype=torch.float32, device=dev),
             "v8": torch.empty(B, H, N, D, dtype=torch.int8, device=dev),
@@ -216,9 +217,9 @@ def rope_rotate_quant_s8(p: Problem, q: Optional[torch.Tensor], k: torch.Tensor,
     rc = lib().ra_rope_rotate_quant_s8(
         C.byref(p), _in_dtype(k), _ptr(q, k.dtype, shp, "q"), _ptr(k, k.dtype, shp, "k"), _ptr(v, k.dtype, shp, "v"),
         _ptr(pos, torch.int32, (N, 3), "pos"),
-        _ptr(out.get("q8") if q is not None else None, torch.int8, shp),
+        _ptr(out.get("q8") if q is not None else None, torch.uint8, shp),
         _ptr(out.get("sq") if q is not None else None, torch.float32, (B, H, N)),
-        _ptr(out["k8"], torch.int8, shp), _ptr(out["sk"], torch.float32, (B, H, N)),
+        _ptr(out["k8"], torch.uint8, shp), _ptr(out["sk"], torch.float32, (B, H, N)),
         _ptr(out["k_mean"], torch.float32, (B, H, D)), _ptr(out["v8"], torch.int8, shp),
         _ptr(out["sv"], torch.float32, (B, H, D)), _ptr(out["v_colsum"], torch.int32, (B, H, _nblocks(p), D)),
         _ptr(workspace, torch.uint8), C.c_size_t(workspace.numel()), C.c_void_p(_stream(stream)))
@@ -234,8 +235,8 @@ def attn_int4_s8(p: Problem, codes: Dict[str, torch.Tensor], out: Optional[torch
     if out is None:
         out = torch.empty(shp, dtype=torch.bfloat16, device=codes["q8"].device)
     rc = lib().ra_attn_int4_s8(
-        C.byref(p), _ptr(codes["q8"], torch.int8, shp), _ptr(codes["sq"], torch.float32, (B, H, N)),
-        _ptr(codes["k8"], torch.int8, shp), _ptr(codes["sk"], torch.float32, (B, H, N)),
+        C.byref(p), _ptr(codes["q8"], torch.uint8, shp), _ptr(codes["sq"], torch.float32, (B, H, N)),
+        _ptr(codes["k8"], torch.uint8, shp), _ptr(codes["sk"], torch.float32, (B, H, N)),
         _ptr(codes["v8"], torch.int8, shp), _ptr(codes["sv"], torch.float32, (B, H, D)),
         _ptr(out, torch.bfloat16, shp, "out"), _ptr(lse, torch.float32, (B, H, N), "lse"),
         C.c_void_p(_stream(stream)))

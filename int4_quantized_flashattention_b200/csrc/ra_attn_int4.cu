@@ -88,6 +88,9 @@ struct Cfg {
   static constexpr int kVwStride = ((kVwBytes + 1023) / 1024) * 1024;
   static constexpr uint32_t kSwz = D == 128 ? kSwizzle128B : kSwizzle64B;
   static constexpr uint32_t kIdescQK = instr_desc(kCfmtS32, 1, 1, 0, 0, kRows, BN);
+  // byte layout: Q and K hold FP8 E4M3 codes, S accumulates in fp32 (exact:
+  // |S_int| <= 49 D < 2^13)
+  static constexpr uint32_t kIdescQKf8 = instr_desc(kCfmtF32, 0, 0, 0, 0, kRows, BN);
   static constexpr uint32_t kIdescPV = instr_desc(kCfmtS32, 0, 1, 0, 1, kRows, D);
   static_assert(D == 64 || D == 128, "head dim");
   static_assert(BN == 16 || BN == 32 || BN == 64, "block_k");
@@ -260,9 +263,11 @@ __device__ __forceinline__ bool wait_at(uint64_t* bar, uint32_t parity, volatile
 // MODE bits 0-1: P codes (0 range-rectified, 1 block-local maximum, 2
 // symmetric); bit 2: fp32 denominator; bit 3: fused Q (warp 3 computes Q's
 // packed codes and scales from the raw Q in place of the TMA load of q4);
-// bit 4: s8 code layout (one code per byte as 16 x code, natural channel
-// order): the TMA loads Q, K and V straight into the MMA operand tiles, and
-// warps 4-7 only stage the per-key scales.
+// bit 4: byte code layout (one code per byte, natural channel order; Q and K
+// as FP8 E4M3 codes, V as 16 x code in s8): the TMA loads Q, K and V straight
+// into the MMA operand tiles, Q K^T runs as kind::f8f6f4 with an fp32 S (no
+// integer conversion in the softmax), and warps 4-7 only stage the per-key
+// scales.
 template <int D, int BN, bool DUMP, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -416,7 +421,8 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           for (int kk = 0; kk < D / 32; ++kk) {
             const uint64_t adesc = smem_desc(sQ + kk * 32, 16, 8 * D, C::kSwz);
             const uint64_t bdesc = smem_desc(sKw + ks * C::kKwStride + kk * 32, 16, 8 * D, C::kSwz);
-            mma_i8_ss(tS, adesc, bdesc, C::kIdescQK, kk > 0 ? 1u : 0u);
+            if constexpr (kS8) mma_f8_ss(tS, adesc, bdesc, C::kIdescQKf8, kk > 0 ? 1u : 0u);
+            else mma_i8_ss(tS, adesc, bdesc, C::kIdescQK, kk > 0 ? 1u : 0u);
           }
           mma_commit(B.s_full + tt * 2 + buf);
           mma_commit(B.kw_empty + ks);
@@ -487,8 +493,7 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
           if (wt < BN) {
             const int j = t * BN + wt;
             float* ksc = reinterpret_cast<float*>(smem + C::oKsc) + ks * BN;
-            ksc[wt] = j < prm.N ? prm.sk[static_cast<size_t>(bh) * prm.N + j] * (1.0f / 256.0f)
-                                : __int_as_float(0x7FC00000);
+            ksc[wt] = j < prm.N ? prm.sk[static_cast<size_t>(bh) * prm.N + j] : __int_as_float(0x7FC00000);
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(B.kw_full + ks);
@@ -678,12 +683,19 @@ attn_int4_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 #pragma unroll
         for (int j = 0; j < kHK; j += 4) {
           const float4 sc = ksc[j / 4];
-          v2[j / 2] = __fmul2_rn(make_float2(static_cast<float>(static_cast<int>(raw[j])),
-                                             static_cast<float>(static_cast<int>(raw[j + 1]))),
-                                 make_float2(sc.x, sc.y));
-          v2[j / 2 + 1] = __fmul2_rn(make_float2(static_cast<float>(static_cast<int>(raw[j + 2])),
-                                                 static_cast<float>(static_cast<int>(raw[j + 3]))),
-                                     make_float2(sc.z, sc.w));
+          if constexpr (kS8) {  // S is already the exact fp32 value of S_int
+            v2[j / 2] = __fmul2_rn(make_float2(__uint_as_float(raw[j]), __uint_as_float(raw[j + 1])),
+                                   make_float2(sc.x, sc.y));
+            v2[j / 2 + 1] = __fmul2_rn(make_float2(__uint_as_float(raw[j + 2]), __uint_as_float(raw[j + 3])),
+                                       make_float2(sc.z, sc.w));
+          } else {
+            v2[j / 2] = __fmul2_rn(make_float2(static_cast<float>(static_cast<int>(raw[j])),
+                                               static_cast<float>(static_cast<int>(raw[j + 1]))),
+                                   make_float2(sc.x, sc.y));
+            v2[j / 2 + 1] = __fmul2_rn(make_float2(static_cast<float>(static_cast<int>(raw[j + 2])),
+                                                   static_cast<float>(static_cast<int>(raw[j + 3]))),
+                                       make_float2(sc.z, sc.w));
+          }
         }
         float vmax = tree_max<kHK>(reinterpret_cast<const float*>(v2));
         vmax = fmaxf(vmax, __shfl_xor_sync(0xFFFFFFFFu, vmax, 16));  // the row's other half

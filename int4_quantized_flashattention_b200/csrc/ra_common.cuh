@@ -240,6 +240,15 @@ __device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint
       ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
 }
 
+// kind::f8f6f4 (A, B FP8 E4M3 in shared memory, D = f32 in TMEM).
+__device__ __forceinline__ void mma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+
 __device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                            uint32_t idesc, uint32_t accumulate) {
   asm volatile(
@@ -278,8 +287,9 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
   return d;
 }
 
-// Instruction descriptor for kind::i8 (D = s32) and kind::f16 (D = f32).
-//   a_fmt/b_fmt: i8 -> 0 unsigned, 1 signed; f16 -> 0 f16, 1 bf16.
+// Instruction descriptor for kind::i8 (D = s32), kind::f16 and kind::f8f6f4
+// (D = f32).  a_fmt/b_fmt: i8 -> 0 unsigned, 1 signed; f16 -> 0 f16, 1 bf16;
+// f8f6f4 -> 0 E4M3.
 __host__ __device__ constexpr uint32_t instr_desc(uint32_t c_fmt, uint32_t a_fmt, uint32_t b_fmt,
                                                   uint32_t a_mn_major, uint32_t b_mn_major,
                                                   uint32_t M, uint32_t N) {

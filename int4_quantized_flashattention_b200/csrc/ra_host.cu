@@ -72,11 +72,11 @@ ra_status ra_rope_rotate_quant(const ra_problem* p, int in_dtype, const void* q,
 }
 
 ra_status ra_rope_rotate_quant_s8(const ra_problem* p, int in_dtype, const void* q, const void* k,
-                                  const void* v, const int32_t* pos, int8_t* q8, float* sq, int8_t* k8,
+                                  const void* v, const int32_t* pos, uint8_t* q8, float* sq, uint8_t* k8,
                                   float* sk, float* k_mean, int8_t* v8, float* sv, int32_t* v_colsum,
                                   void* workspace, size_t ws_bytes, void* stream) {
-  return rope_rotate_quant(p, in_dtype, q, k, v, pos, reinterpret_cast<uint8_t*>(q8), sq,
-                           reinterpret_cast<uint8_t*>(k8), sk, k_mean, reinterpret_cast<uint8_t*>(v8), sv, v_colsum,
+  return rope_rotate_quant(p, in_dtype, q, k, v, pos, q8, sq, k8, sk, k_mean, reinterpret_cast<uint8_t*>(v8), sv,
+                           v_colsum,
                            workspace, ws_bytes, stream, true);
 }
 
@@ -96,7 +96,7 @@ static ra_status rope_rotate_quant(const ra_problem* p, int in_dtype, const void
                                        workspace, static_cast<cudaStream_t>(stream), s8));
 }
 
-ra_status ra_attn_int4_s8(const ra_problem* p, const int8_t* q8, const float* sq, const int8_t* k8,
+ra_status ra_attn_int4_s8(const ra_problem* p, const uint8_t* q8, const float* sq, const uint8_t* k8,
                           const float* sk, const int8_t* v8, const float* sv, void* out, float* lse,
                           void* stream) {
   if (!valid_problem(p)) return RA_ERR_INVALID_ARG;
@@ -106,9 +106,8 @@ ra_status ra_attn_int4_s8(const ra_problem* p, const int8_t* q8, const float* sq
   if (!aligned16_or_null(lse)) return RA_ERR_INVALID_ARG;
   if (p->block_k != 64) return RA_ERR_UNSUPPORTED;
   int unsupported = 0;
-  cudaError_t e = ra::launch_attn_int4(*p, reinterpret_cast<const uint8_t*>(q8), sq,
-                                       reinterpret_cast<const uint8_t*>(k8), sk,
-                                       reinterpret_cast<const uint8_t*>(v8), sv, out, lse, nullptr, 16,
+  cudaError_t e = ra::launch_attn_int4(*p, q8, sq, k8, sk, reinterpret_cast<const uint8_t*>(v8), sv, out, lse,
+                                       nullptr, 16,
                                        static_cast<cudaStream_t>(stream), &unsupported);
   if (unsupported) return RA_ERR_UNSUPPORTED;
   return from_cuda(e);

@@ -97,10 +97,10 @@ struct PrologueArgs {
   double* ksum;     // [BH, nchunk, D]
   float* vmax;      // [BH, nchunk, D]
   float* vinv;      // [BH, D]
-  uint8_t *q4, *k4, *v4;   // packed codes [BH, N, D/2], or s8 codes [BH, N, D] when s8
+  uint8_t *q4, *k4, *v4;   // packed codes [BH, N, D/2], or bytes [BH, N, D] when s8 (Q, K: E4M3 codes; V: 16 x code)
   float *sq, *sk, *k_mean, *sv;
   int32_t* colsum;
-  int s8;                  // code layout: 0 packed nibbles, 1 one code per byte (16 x code)
+  int s8;                  // code layout: 0 packed nibbles, 1 one code per byte
 };
 
 // Table entry e -> (segment j, position g, pair k); angle g * theta^(-2k/Dj) in
@@ -444,8 +444,8 @@ __global__ void __launch_bounds__(kThreads, 3) prologue_quant_kernel(PrologueArg
         const size_t o4 = head4 + static_cast<size_t>(n) * (kD / 2) + (c0 >> 1);
         if constexpr (kS8) {
           const size_t o8 = head + static_cast<size_t>(n) * kD + c0;
-          if constexpr (kQ) *reinterpret_cast<uint2*>(a.q4 + o8) = make_uint2(pack4_s8_bits(bq), pack4_s8_bits(bq + 4));
-          *reinterpret_cast<uint2*>(a.k4 + o8) = make_uint2(pack4_s8_bits(bk), pack4_s8_bits(bk + 4));
+          if constexpr (kQ) *reinterpret_cast<uint2*>(a.q4 + o8) = make_uint2(pack4_e4m3_bits(bq), pack4_e4m3_bits(bq + 4));
+          *reinterpret_cast<uint2*>(a.k4 + o8) = make_uint2(pack4_e4m3_bits(bk), pack4_e4m3_bits(bk + 4));
           *reinterpret_cast<uint2*>(a.v4 + o8) = make_uint2(pack4_s8_bits(bv), pack4_s8_bits(bv + 4));
         } else {
           if constexpr (kQ) *reinterpret_cast<uint32_t*>(a.q4 + o4) = pack8_bits(bq);

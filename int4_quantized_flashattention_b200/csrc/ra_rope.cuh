@@ -238,8 +238,8 @@ __device__ __forceinline__ uint32_t pack8_bits(const uint32_t* b) {
   return (acc - kQBitsRep) ^ 0x88888888u;
 }
 
-// The s8 code layout: one code per byte, held in the byte's high nibble (the
-// s8 value 16 x code, the low nibble zero), channels in natural order.  For
+// The byte code layout (V): one code per byte, held in the byte's high nibble
+// (the s8 value 16 x code, the low nibble zero), channels in natural order.  For
 // four quant4_bits2 results b[0..3] (channels c..c+3) the little-endian word
 // of their bytes: sum_i 256^i b_i minus the known offsets leaves the bytes
 // code + 8 (at most 15: no carries), shifted into the high nibble; XOR 0x80
@@ -251,6 +251,20 @@ __device__ __forceinline__ uint32_t pack4_s8_bits(const uint32_t* b) {
   acc = acc * 256u + b[1];
   acc = acc * 256u + b[0];
   return ((acc - kQBitsRep4) << 4) ^ 0x80808080u;
+}
+
+// FP8 E4M3 bytes of four codes (channels c..c+3, little-endian) from their
+// quant4_bits2 results: the code as a float is the bits' value minus
+// 1.5 * 2^23 + 8 (exact), and every integer in [-7, 7] is exact in E4M3.
+__device__ __forceinline__ uint32_t pack4_e4m3_bits(const uint32_t* b) {
+  float c[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) c[i] = __fsub_rn(__uint_as_float(b[i]), kQMagic8);
+  uint16_t lo, hi;
+  // the first source goes to the upper byte of each pair
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(c[1]), "f"(c[0]));
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(c[3]), "f"(c[2]));
+  return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
 }
 
 // Max over the D/8 threads of a token (a contiguous lane group of size lpt).

@@ -1,8 +1,10 @@
-"""The s8 code layout (ra_rope_rotate_quant_s8 / ra_attn_int4_s8): one code
-per byte as 16 x code, natural channel order, loaded by TMA straight into the
-MMA operand tiles.  The codes must be the packed prologue's codes (times 16)
-bit for bit, every other prologue output identical, and the attention's out
-and lse identical to ra_attn_int4 on the packed codes; the packed path is
+"""The byte code layout (ra_rope_rotate_quant_s8 / ra_attn_int4_s8): one code
+per byte, natural channel order (Q and K as FP8 E4M3 values equal to the
+code, V as the int8 value 16 x code), loaded by TMA straight into the MMA
+operand tiles; Q K^T runs in FP8 with an fp32 accumulator.  The codes must be
+the packed prologue's codes bit for bit, every other prologue output
+identical, and the attention's out and lse identical to ra_attn_int4 on the
+packed codes (which also shows the FP8 Q K^T is exact); the packed path is
 checked against the oracle in test_gpu_int4.py.
 """
 import numpy as np
@@ -27,6 +29,22 @@ def _unpack16(packed):
     return (oracle.unpack_codes(packed).astype(np.int16) * 16).astype(np.int8)
 
 
+def _e4m3(c):
+    """FP8 E4M3 byte of each integer code in [-7, 7] (sign, 4 exponent bits
+    with bias 7, 3 mantissa bits), written out from the format's definition."""
+    c = np.asarray(c, np.int64)
+    a = np.abs(c)
+    e = np.floor(np.log2(np.maximum(a, 1))).astype(np.int64)
+    m = ((a / np.exp2(e) - 1.0) * 8).astype(np.int64)
+    byte = np.where(a == 0, 0, ((e + 7) << 3) | m) | np.where(c < 0, 0x80, 0)
+    return byte.astype(np.uint8)
+
+
+def test_e4m3_table():
+    assert list(_e4m3(np.arange(-7, 8))) == [0xCE, 0xCC, 0xCA, 0xC8, 0xC4, 0xC0, 0xB8, 0x00,
+                                             0x38, 0x40, 0x44, 0x48, 0x4A, 0x4C, 0x4E]
+
+
 def _run(ra, wl):
     import torch
     dev = gu.device()
@@ -39,10 +57,13 @@ def _run(ra, wl):
     assert ra.sync_status() == 0
     s8 = ra.rope_rotate_quant_s8(p, q, k, v, pos)
     assert ra.sync_status() == 0
-    for a, b in (("q8", "q4"), ("k8", "k4"), ("v8", "v4")):
+    import oracle
+    for a, b in (("q8", "q4"), ("k8", "k4")):
         got = s8[a].cpu().numpy().reshape(-1, wl.D)
-        ref = _unpack16(packed[b].cpu().numpy().reshape(-1, wl.D // 2))
+        ref = _e4m3(oracle.unpack_codes(packed[b].cpu().numpy().reshape(-1, wl.D // 2)))
         assert np.array_equal(got, ref), a
+    got = s8["v8"].cpu().numpy().reshape(-1, wl.D)
+    assert np.array_equal(got, _unpack16(packed["v4"].cpu().numpy().reshape(-1, wl.D // 2)))
     for name in ("sq", "sk", "k_mean", "sv", "v_colsum"):
         assert torch.equal(s8[name], packed[name]), name
     out = torch.full_like(out_ref, float("nan"))
