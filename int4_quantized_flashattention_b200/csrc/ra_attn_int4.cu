@@ -31,6 +31,10 @@
 //     TMA producer, two MMA issuers, four widening warps and 16 softmax warps
 //     (two threads per query row, each with half of the keys of a block and
 //     half of the output columns).  Persistent CTAs, one per SM.
+//   * Variants (MODE bits): the ablation switches; fused Q (warp 3 produces
+//     each item's packed Q from the raw Q); the byte code layout (Q, K as FP8
+//     E4M3 codes and V as 16 x code, TMA'd straight into the operand tiles, an
+//     FP8 Q K^T with an exact fp32 S, no widening).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>

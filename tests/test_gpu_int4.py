@@ -380,8 +380,8 @@ def test_dump_variant_matches_production_bitwise(ra, dev, orc, D, seg, grid, p_m
         assert np.array_equal(lse.cpu().numpy(), host["lse"]), (h, tile)
 
 
-@pytest.mark.parametrize("name", ["sweep8192", "sweep8192_half", "sweep16384", "sweep16384_half",
-                                  "sweep32760_half", "sweep65536", "sweep65536_half"])
+@pytest.mark.parametrize("name", ["sweep4096", "sweep4096_half", "sweep8192", "sweep8192_half", "sweep16384",
+                                  "sweep16384_half", "sweep32760_half", "sweep65536", "sweep65536_half"])
 def test_sweep_sampled(ra, dev, orc, name):
     """The sweep shapes (H = 40, D = 128) at full size in both rotation modes:
     the prologue of two heads in full, and the first, middle and last (for
