@@ -49,3 +49,26 @@ def test_traffic_is_reported_only_for_the_measured_sources(tmp_path, monkeypatch
     (tmp_path / "int4_quantized_flashattention_b200" / "csrc" / "ra_attn_int4.cu").write_bytes(b"kernel v2")
     assert bench._attn_traffic() is None
 
+
+
+def test_launch_count_per_step_by_rotation_mode():
+    """The interleaved rotation builds two RoPE tables (the fused one and the
+    plain one of the channel reduce), the other modes one: reduce, finalize,
+    quantise and the attention make the rest."""
+    assert bench.kernels_per_step(1) == 6
+    for rot in (0, 2, 3):
+        assert bench.kernels_per_step(rot) == 5
+
+
+def test_reference_arm_marks_its_time_as_extrapolated():
+    """--impl reference on a small workload: the line carries the sample's own
+    time beside the extrapolated step time, and the e2e object the contract
+    asks for (no host-device copies)."""
+    import argparse
+    args = argparse.Namespace(workload="tiny", block_k=None, steps=1, warmup=3, ref_seconds=1.0)
+    r = bench.run_reference(args)
+    assert r["impl"] == "reference" and r["extrapolated"] is True
+    assert r["sample_ms_per_step"] > 0 and r["ms_per_step"] > 0
+    assert r["cpu_baseline"]["kind"] == "oracle" and r["cpu_baseline"]["cores"] >= 1
+    assert r["e2e"]["h2d_bytes_per_step"] == 0 and r["e2e"]["d2h_bytes_per_step"] == 0
+    assert r["e2e"]["value"] == r["value"]
