@@ -460,7 +460,7 @@ def run_ours(args, rank, world, local_rank):
         "e2e": {"value": round(weak_scaling_value(world, ops, e2e_ms), 2), "unit": "TOPS",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4),
                 "copies": "H2D and D2H on their own streams, overlapping the previous and next steps' kernels"},
-        "roofline": {"bound": "tensor", "kernel": "attn_int4_kernel", "achieved": round(achieved, 1),
+        "roofline": {"bound": "tensor", "kernel": "attn_int4_pair_kernel" if wl.block_k == 128 else "attn_int4_kernel", "achieved": round(achieved, 1),
                      "peak": round(int8_peak, 1), "unit": "TFLOP/s", "frac": round(achieved / int8_peak, 4),
                      "peak_source": f"2 x {pk['source']} bf16 burst {pk['bf16_tflops']} TFLOP/s (int8 ops/s)",
                      "traffic": _attn_traffic() if (args.workload == "wan" and args.block_k is None) else None},
