@@ -66,6 +66,12 @@ def _run(ra, wl):
     assert np.array_equal(got, _unpack16(packed["v4"].cpu().numpy().reshape(-1, wl.D // 2)))
     for name in ("sq", "sk", "k_mean", "sv", "v_colsum"):
         assert torch.equal(s8[name], packed[name]), name
+    # K and V only (q = None): the same K and V outputs, nothing for Q
+    kv = ra.rope_rotate_quant_s8(p, None, k, v, pos)
+    assert ra.sync_status() == 0
+    assert set(kv) == {"k8", "sk", "k_mean", "v8", "sv", "v_colsum"}
+    for name, t in kv.items():
+        assert torch.equal(t, s8[name]), name
     out = torch.full_like(out_ref, float("nan"))
     lse = torch.full_like(lse_ref, float("nan"))
     ra.attn_int4_s8(p, s8, out=out, lse=lse)
